@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""Benchmark of Dynamic Bifocal RoPE attention on B200.
+
+One step = one bifocal causal prefill of a 131072-token sequence (32 query / 8
+KV heads, head_dim 128, w_pretrained 32768 so G = 4, w0 4096, bf16) followed
+by the 256 decode steps of the decode workload (a 131072..131327-token
+standard-RoPE cache, G recomputed every step: 4, then 5).  Inputs are seeded
+synthetic tensors already resident in HBM; every input is larger than L2, so
+no flush is needed between iterations.
+
+metric / value: prefill TFLOP/s, algorithmic FLOPs 4 * D * Hq * sum L(L+1)/2
+(causal QK^T + PV only) over the prefill's device time.  The decode part is
+reported under "decode" (us/token and HBM GB/s, K+V bytes 2 * L * Hkv * D * 2
+per step).
+
+python bench.py --gpus N --steps K --warmup W [--impl reference]
+Under torchrun (N > 1) every rank runs an independent replica ("replicas
+only": the path has no exchange step); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from zero_shot_rope_b200 import synth  # noqa: E402
+
+METRIC = "bifocal prefill TFLOP/s @128K (frac of bf16 peak); decode µs/tok + HBM GB/s"
+PREFILL = "prefill_128k_g4"
+DECODE = "decode_128k"
+
+
+def prefill_flops(w) -> float:
+    D, Hq = w.head_dim, w.n_q_heads
+    return float(sum(4.0 * D * Hq * L * (L + 1) / 2 for L in w.seqlens))
+
+
+def rows_flops(w, rows) -> float:
+    # algorithmic FLOPs of the given query rows (positions) over all heads
+    return float(sum(4.0 * w.head_dim * w.n_q_heads * (int(r) + 1) for r in rows))
+
+
+def decode_bytes(w, L) -> int:
+    return 2 * L * w.n_kv_heads * w.head_dim * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_traffic(name):
+    """DRAM bytes per launch from the committed ncu summary, valid only while
+    the kernel source is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(name)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return d["bytes_per_launch"] if sha == d["source_sha"] else None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = os.path.join("/tmp", f"jl_clocks_{os.getpid()}.csv")
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                if self.uuid and self.uuid.replace("GPU-", "") not in parts[1]:
+                    continue
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[6:10]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample_rows(w, n, seed):
+    rng = np.random.default_rng(seed)
+    L = w.seqlens[0]
+    return np.sort(rng.choice(np.arange(w.w0, L), size=n, replace=False))
+
+
+def cpu_oracle(w, q, k, v, cu, rows):
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    t0 = time.perf_counter()
+    oracle.bifocal_attention(q, k, v, cu, w.w_pretrained, w.w0, w.rope_theta, rows=rows)
+    dt = time.perf_counter() - t0
+    return dt, threads
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the fp64 CPU oracle as it stands, on a bounded sample."""
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[PREFILL]
+    q, k, v, cu = synth.prefill_inputs(w)
+    n_rows = args.ref_rows
+    times = []
+    threads = 1
+    for s in range(args.warmup + args.steps):
+        rows = oracle_sample_rows(w, n_rows, seed=s)
+        dt, threads = cpu_oracle(w, q, k, v, cu, rows)
+        if s >= args.warmup:
+            times.append((dt, rows_flops(w, rows)))
+    tot_t = sum(t for t, _ in times)
+    tot_f = sum(f for _, f in times)
+    value = tot_f / tot_t / 1e12
+    sample = f"{n_rows} query rows x {w.n_q_heads} heads of the {w.seqlens[0]}-token prefill per step (fp64 oracle)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "seq_len": w.seqlens[0],
+                                        "heads": f"{w.n_q_heads}/{w.n_kv_heads}", "head_dim": w.head_dim,
+                                        "G": 4, "w0": w.w0},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    from zero_shot_rope_b200 import jetlong as jl
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wp = synth.WORKLOADS[PREFILL]
+    wd = synth.WORKLOADS[DECODE]
+    peaks, peak_kind = load_peaks()
+
+    # ---- inputs (seeded CPU draws, then resident in HBM)
+    q_h, k_h, v_h, cu_h = synth.prefill_inputs(wp)
+    q, k, v, cu = q_h.to(dev), k_h.to(dev), v_h.to(dev), cu_h.to(dev)
+    out = torch.empty_like(q)
+    T = wp.total_tokens
+    ws_p = torch.empty(jl.jl_bifocal_prefill_workspace_size(1, T, wp.n_q_heads, wp.n_kv_heads, wp.head_dim),
+                       dtype=torch.uint8, device=dev)
+    kc_h, vc_h = synth.decode_cache(wd)
+    kc, vc = kc_h.to(dev), vc_h.to(dev)
+    n_dec = args.decode_steps
+    cap = kc.shape[1]
+    qd_h = torch.stack([synth.decode_query(wd, t) for t in range(n_dec)])  # [n, 1, Hq, D]
+    qd = qd_h.to(dev)
+    od = torch.empty_like(qd)
+    lens = torch.tensor([wd.seqlens[0] + t for t in range(n_dec)], dtype=torch.int32, device=dev)
+    ws_d = torch.empty(jl.jl_bifocal_decode_workspace_size(1, wd.n_q_heads, wd.n_kv_heads, wd.head_dim, cap),
+                       dtype=torch.uint8, device=dev)
+    pf_flops = prefill_flops(wp)
+    dec_bytes = sum(decode_bytes(wd, wd.seqlens[0] + t) for t in range(n_dec))
+
+    def prefill(flags=0):
+        jl.jl_bifocal_prefill(q, k, v, cu, T, wp.w_pretrained, wp.w0, wp.rope_theta, out=out, flags=flags,
+                              workspace=ws_p)
+
+    def decode_all(flags=0):
+        for t in range(n_dec):
+            jl.jl_bifocal_decode(qd[t], kc, vc, lens[t:t + 1], cap, wd.w_pretrained, wd.w0, wd.rope_theta,
+                                 out=od[t], flags=flags, workspace=ws_d)
+
+    # ---- warm-up
+    for _ in range(args.warmup):
+        prefill()
+        decode_all()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, device-resident inputs
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for s in range(args.steps):
+        ev[s][0].record()
+        prefill()
+        ev[s][1].record()
+        decode_all()
+        ev[s][2].record()
+    t_end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    pre_ms_max = max_over_ranks(sum(pre_ms), world, dev)
+    dec_ms_max = max_over_ranks(sum(dec_ms), world, dev)
+    value = world * args.steps * pf_flops / (pre_ms_max * 1e-3) / 1e12
+    launches_per_step = 2 + 2 * n_dec  # prefill: pre-rotation + attention; decode: partial + combine
+
+    # ---- plain-causal comparison (outside the timed region)
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record()
+    prefill(jl.JL_FLAG_PLAIN_CAUSAL)
+    e1.record()
+    decode_all(jl.JL_FLAG_PLAIN_CAUSAL)
+    e2.record()
+    torch.cuda.synchronize()
+    plain_pre_ms, plain_dec_ms = e0.elapsed_time(e1), e1.elapsed_time(e2)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        qp, kp, vp = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        outp = torch.empty(q_h.shape, dtype=q_h.dtype).pin_memory()
+        qdp = qd_h.pin_memory()
+        odp = torch.empty(qd_h.shape, dtype=qd_h.dtype).pin_memory()
+        h2d = (qp.numel() + kp.numel() + vp.numel()) * 2 + qdp.numel() * 2
+        d2h = outp.numel() * 2 + odp.numel() * 2
+
+        def e2e_step():
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            prefill()
+            outp.copy_(out, non_blocking=True)
+            for t in range(n_dec):
+                qd[t].copy_(qdp[t], non_blocking=True)
+                jl.jl_bifocal_decode(qd[t], kc, vc, lens[t:t + 1], cap, wd.w_pretrained, wd.w0, wd.rope_theta,
+                                     out=od[t], workspace=ws_d)
+                odp[t].copy_(od[t], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record()
+        pre_e2e = []
+        for _ in range(args.steps):
+            b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b0.record()
+            q.copy_(qp, non_blocking=True)
+            k.copy_(kp, non_blocking=True)
+            v.copy_(vp, non_blocking=True)
+            prefill()
+            outp.copy_(out, non_blocking=True)
+            b1.record()
+            pre_e2e.append((b0, b1))
+            for t in range(n_dec):
+                qd[t].copy_(qdp[t], non_blocking=True)
+                jl.jl_bifocal_decode(qd[t], kc, vc, lens[t:t + 1], cap, wd.w_pretrained, wd.w0, wd.rope_theta,
+                                     out=od[t], workspace=ws_d)
+                odp[t].copy_(od[t], non_blocking=True)
+        a1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        pre_e2e_ms = max_over_ranks(sum(b0.elapsed_time(b1) for b0, b1 in pre_e2e), world, dev)
+        e2e = {"value": world * args.steps * pf_flops / (pre_e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": max_over_ranks(a0.elapsed_time(a1), world, dev) / args.steps}
+
+    # ---- CPU baseline (rank 0, N = 1 only): the oracle on a bounded sample
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = oracle_sample_rows(wp, args.cpu_rows, seed=123)
+        dt, threads = cpu_oracle(wp, q_h, k_h, v_h, cu_h, rows)
+        cpu = {"value": rows_flops(wp, rows) / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{len(rows)} random query rows x {wp.n_q_heads} heads of the {wp.seqlens[0]}-token "
+                         f"prefill (fp64 NumPy oracle, {dt:.1f} s)"}
+
+    if rank != 0:
+        return
+    mean_pre_ms = statistics.mean(pre_ms)
+    achieved = pf_flops / (mean_pre_ms * 1e-3) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    dec_us_tok = 1e3 * statistics.mean(dec_ms) / n_dec
+    dec_gbs = dec_bytes / (statistics.mean(dec_ms) * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{wp.name} + {wd.name}", "seq_len": wp.seqlens[0],
+                   "heads": f"{wp.n_q_heads}/{wp.n_kv_heads}", "head_dim": wp.head_dim,
+                   "w_pretrained": wp.w_pretrained, "G": 4, "w0": wp.w0, "rope_theta": wp.rope_theta,
+                   "decode_steps": n_dec, "decode_L": [wd.seqlens[0], wd.seqlens[0] + n_dec - 1],
+                   "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush needed)"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": kernel_traffic("bifocal_prefill_kernel"),
+                     "kernel": "jl_bifocal_prefill (pre-rotation + tcgen05 attention kernel)",
+                     "peak_kind": f"{peak_kind} bf16 sustained",
+                     "frac_of_burst_peak": achieved / peaks["bf16_tflops"]},
+        "decode": {"us_per_tok": dec_us_tok, "hbm_gbs": dec_gbs, "hbm_peak_gbs": peaks["hbm_gbs"],
+                   "frac": dec_gbs / peaks["hbm_gbs"], "bytes_per_step": dec_bytes / n_dec,
+                   "plain_us_per_tok": 1e3 * plain_dec_ms / n_dec,
+                   "overhead_vs_plain": (statistics.mean(dec_ms) - plain_dec_ms) / plain_dec_ms},
+        "prefill": {"ms": mean_pre_ms, "plain_ms": plain_pre_ms,
+                    "plain_tflops": pf_flops / (plain_pre_ms * 1e-3) / 1e12,
+                    "bifocal_over_plain_time": mean_pre_ms / plain_pre_ms},
+        "clocks": clk,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--cpu-rows", type=int, default=24)
+    ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            from zero_shot_rope_b200 import build
+
+            if rank == 0:
+                build.build()
+            barrier(world)
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

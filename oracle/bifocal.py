@@ -144,11 +144,12 @@ def _seq_bounds(cu_seqlens):
 # ---------------------------------------------------------------------------
 
 
-def _attend_rows_direct(q_rows, pos_i, K, V, L, G, w0, theta, plain):
+def _attend_rows_direct(q_rows, pos_i, K, K_g, V, G, w0, theta, plain):
     """Scores of query rows against keys 0..L-1 of one sequence and one head.
 
     q_rows [R, D] standard-RoPE queries at positions pos_i; K [L, D]
-    standard-RoPE keys at positions 0..L-1; V [L, D].
+    standard-RoPE keys at positions 0..L-1; K_g [L, D] the same keys rotated
+    by R(delta(p_j)) (None when ``plain``); V [L, D].
 
     For each pair with 0 <= d = p_i - p_j:
       d <  w0  ->  s = <Q~_i, K~_j> / sqrt(D)                       (local, base RoPE)
@@ -156,7 +157,7 @@ def _attend_rows_direct(q_rows, pos_i, K, V, L, G, w0, theta, plain):
     "Janela Local" / "Janela Remota" bullets of §1 and the correction rotation
     of §2.  ``plain`` scores every pair with the base RoPE (G irrelevant).
     """
-    D = K.shape[1]
+    L, D = K.shape
     scale = 1.0 / math.sqrt(D)
     pos_j = np.arange(L, dtype=np.int64)
     dist = pos_i[:, None] - pos_j[None, :]
@@ -165,24 +166,32 @@ def _attend_rows_direct(q_rows, pos_i, K, V, L, G, w0, theta, plain):
         S = S_std
     else:
         q_g = rope_rotate(q_rows, correction_shift(pos_i, G), theta)
-        k_g = rope_rotate(K, correction_shift(pos_j, G), theta)
-        S_grp = (q_g @ k_g.T) * scale
+        S_grp = (q_g @ K_g.T) * scale
         S = np.where(dist < w0, S_std, S_grp)
     S = np.where(dist >= 0, S, -np.inf)
     return _softmax_rows(S, V)
+
+
+def _take64(t, idx, h):
+    """fp64 copy of t[idx, h] for a torch tensor or a numpy array."""
+    if hasattr(t, "detach"):
+        import torch
+
+        return _as64(t[torch.as_tensor(np.asarray(idx, dtype=np.int64)), h])
+    return np.asarray(t[np.asarray(idx), h], dtype=np.float64)
 
 
 def bifocal_attention(q, k, v, cu_seqlens, w_pretrained, w0, theta, rows=None, plain=False,
                       row_batch=64):
     """Dynamic Bifocal RoPE causal GQA prefill attention, route A (direct).
 
-    q [T, Hq, D], k/v [T, Hkv, D] (any float type; computed in fp64), packed by
-    ``cu_seqlens`` [B+1]; query head h reads kv head h // (Hq / Hkv).
+    q [T, Hq, D], k/v [T, Hkv, D] (any float type, torch or numpy; computed in
+    fp64), packed by ``cu_seqlens`` [B+1]; query head h reads kv head
+    h // (Hq / Hkv).
 
     ``rows``: optional sorted global token indices to evaluate (default: all).
     Returns (out [len(rows), Hq, D], lse [Hq, len(rows)]) in fp64.
     """
-    q, k, v = _as64(q), _as64(k), _as64(v)
     T, Hq, D = q.shape
     Hkv = k.shape[1]
     group = Hq // Hkv
@@ -195,15 +204,19 @@ def bifocal_attention(q, k, v, cu_seqlens, w_pretrained, w0, theta, rows=None, p
         if L == 0 or len(sel) == 0:
             continue
         G = group_size(L, w_pretrained)
-        for h in range(Hq):
-            kv = h // group
-            K, V = k[a:b, kv], v[a:b, kv]
-            for c in range(0, len(sel), row_batch):
-                idx = sel[c:c + row_batch]
-                pos_i = rows[idx] - a
-                o, l_ = _attend_rows_direct(q[rows[idx], h], pos_i, K, V, L, G, w0, theta, plain)
-                out[idx, h] = o
-                lse[h, idx] = l_
+        pos_j = np.arange(L, dtype=np.int64)
+        for kv in range(Hkv):
+            K = _take64(k, np.arange(a, b), kv)
+            V = _take64(v, np.arange(a, b), kv)
+            K_g = None if plain else rope_rotate(K, correction_shift(pos_j, G), theta)
+            for h in range(kv * group, (kv + 1) * group):
+                for c in range(0, len(sel), row_batch):
+                    idx = sel[c:c + row_batch]
+                    pos_i = rows[idx] - a
+                    o, l_ = _attend_rows_direct(_take64(q, rows[idx], h), pos_i, K, K_g, V, G, w0,
+                                                theta, plain)
+                    out[idx, h] = o
+                    lse[h, idx] = l_
     return out, lse
 
 
@@ -229,15 +242,16 @@ def bifocal_decode(q, k_cache, v_cache, seqlens, w_pretrained, w0, theta, plain=
         if L == 0:
             continue
         G = group_size(L, w_pretrained)
-        K_all = _as64(k_cache[b, :L])
-        V_all = _as64(v_cache[b, :L])
         pos_i = np.array([L - 1], dtype=np.int64)
-        for h in range(Hq):
-            kv = h // group
-            o, l_ = _attend_rows_direct(q[b, h][None, :], pos_i, K_all[:, kv], V_all[:, kv], L, G,
-                                        w0, theta, plain)
-            out[b, h] = o[0]
-            lse[b, h] = l_[0]
+        pos_j = np.arange(L, dtype=np.int64)
+        for kv in range(Hkv):
+            K = _as64(k_cache[b, :L, kv])
+            V = _as64(v_cache[b, :L, kv])
+            K_g = None if plain else rope_rotate(K, correction_shift(pos_j, G), theta)
+            for h in range(kv * group, (kv + 1) * group):
+                o, l_ = _attend_rows_direct(q[b, h][None, :], pos_i, K, K_g, V, G, w0, theta, plain)
+                out[b, h] = o[0]
+                lse[b, h] = l_[0]
     return out, lse
 
 

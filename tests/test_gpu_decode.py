@@ -1,0 +1,91 @@
+"""Decode parity on the GPU: the split-KV kernel (through the C ABI) against
+the fp64 oracle at every tested step."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from zero_shot_rope_b200 import synth
+from tests.gpu_util import assert_close, jl, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def decode_gpu(q, kc, vc, seqlens, max_seqlen, w_pre, w0, theta, flags=0):
+    J = jl()
+    dev = torch.device("cuda:0")
+    B, Hq, _ = q.shape
+    lse = torch.full((B, Hq), float("nan"), dtype=torch.float32, device=dev)
+    out, lse = J.jl_bifocal_decode(q.to(dev), kc.to(dev), vc.to(dev),
+                                   torch.tensor(seqlens, dtype=torch.int32, device=dev), max_seqlen,
+                                   w_pre, w0, theta, lse=lse, flags=flags)
+    torch.cuda.synchronize()
+    return out, lse
+
+
+SMALL = [
+    # (seqlens, cap, Hq, Hkv, D, w_pre, w0, dtype)
+    ((1,), 8, 4, 1, 128, 1, 0, torch.bfloat16),
+    ((100,), 128, 8, 2, 128, 40, 16, torch.bfloat16),
+    ((1000,), 1024, 32, 8, 128, 250, 64, torch.bfloat16),       # G = 4
+    ((1001,), 1024, 32, 8, 128, 250, 64, torch.bfloat16),       # G = 5 (just crossed)
+    ((3333, 17, 2048), 4000, 16, 8, 128, 700, 300, torch.bfloat16),
+    ((5000,), 5000, 8, 8, 128, 900, 0, torch.bfloat16),
+    ((600,), 700, 8, 1, 128, 100, 600, torch.bfloat16),          # all keys local
+    ((700,), 700, 4, 2, 64, 150, 50, torch.bfloat16),
+    ((900, 33), 1000, 4, 4, 64, 200, 10, torch.float32),
+    ((2500,), 2600, 16, 2, 128, 512, 100, torch.float32),
+]
+
+
+@pytest.mark.parametrize("seqlens,cap,Hq,Hkv,D,w_pre,w0,dtype", SMALL)
+def test_decode_small_cases(seqlens, cap, Hq, Hkv, D, w_pre, w0, dtype):
+    B = len(seqlens)
+    g = torch.Generator().manual_seed(sum(seqlens) + D)
+    q = torch.randn(B, Hq, D, generator=g).to(dtype)
+    kc = torch.randn(B, cap, Hkv, D, generator=g).to(dtype)
+    vc = torch.randn(B, cap, Hkv, D, generator=g).to(dtype)
+    out, lse = decode_gpu(q, kc, vc, list(seqlens), max(seqlens), w_pre, w0, 1e6)
+    ro, rl = oracle.bifocal_decode(q, kc, vc, list(seqlens), w_pre, w0, 1e6)
+    assert_close(to_np(out), ro, dtype, "out")
+    assert_close(to_np(lse), rl, dtype, "lse")
+    po, pl = decode_gpu(q, kc, vc, list(seqlens), max(seqlens), w_pre, w0, 1e6,
+                        flags=jl().JL_FLAG_PLAIN_CAUSAL)
+    rpo, rpl = oracle.bifocal_decode(q, kc, vc, list(seqlens), w_pre, w0, 1e6, plain=True)
+    assert_close(to_np(po), rpo, dtype, "plain out")
+
+
+@pytest.fixture(scope="module")
+def decode_cache():
+    w = synth.WORKLOADS["decode_128k"]
+    kc, vc = synth.decode_cache(w)
+    return w, kc, vc
+
+
+@pytest.mark.parametrize("step", [0, 1, 2, 255])
+def test_decode_128k_steps(decode_cache, step):
+    """Full-size decode in the benchmark's launch configuration: G = 4 at the
+    first step, 5 afterwards (the cache never changes)."""
+    w, kc, vc = decode_cache
+    L = w.seqlens[0] + step
+    q = synth.decode_query(w, step)
+    cap = kc.shape[1]
+    out, lse = decode_gpu(q, kc, vc, [L], cap, w.w_pretrained, w.w0, w.rope_theta)
+    ro, rl = oracle.bifocal_decode(q, kc, vc, [L], w.w_pretrained, w.w0, w.rope_theta)
+    assert_close(to_np(out), ro, torch.bfloat16, f"step {step}")
+    assert_close(to_np(lse), rl, torch.bfloat16, f"step {step} lse")
+    got = to_np(out)
+    assert np.linalg.norm(got - ro) / np.linalg.norm(ro) < 1e-2
+    po, _ = oracle.bifocal_decode(q, kc, vc, [L], w.w_pretrained, w.w0, w.rope_theta, plain=True)
+    assert np.abs(po - ro).mean() > 5 * np.abs(got - ro).mean()
+
+
+def test_decode_zero_length_writes_zero():
+    dev = torch.device("cuda:0")
+    q = torch.randn(2, 8, 128).to(torch.bfloat16)
+    kc = torch.randn(2, 64, 2, 128).to(torch.bfloat16)
+    vc = torch.randn(2, 64, 2, 128).to(torch.bfloat16)
+    out, lse = decode_gpu(q, kc, vc, [0, 50], 64, 16, 8, 1e4)
+    assert torch.all(out[0] == 0) and torch.all(torch.isinf(lse[0]))
+    ro, _ = oracle.bifocal_decode(q[1:], kc[1:], vc[1:], [50], 16, 8, 1e4)
+    assert_close(to_np(out[1:]), ro, torch.bfloat16, "row 1")

@@ -1,0 +1,104 @@
+"""Prefill parity on the GPU: the CUDA path (through the C ABI) against the
+fp64 oracle, element by element, plus bitwise invariants between modes."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from zero_shot_rope_b200 import synth
+from tests.gpu_util import assert_close, jl, prefill_gpu, sample_rows, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_fp32_workload_full():
+    w = synth.WORKLOADS["tiny_fp32"]
+    q, k, v, cu = synth.prefill_inputs(w)
+    out, lse = prefill_gpu(q, k, v, cu, w.w_pretrained, w.w0, w.rope_theta)
+    ro, rl = oracle.bifocal_attention(q, k, v, cu, w.w_pretrained, w.w0, w.rope_theta)
+    assert_close(to_np(out), ro, torch.float32, "out")
+    assert_close(to_np(lse), rl, torch.float32, "lse")
+
+
+CASES = [
+    # (seqlens, Hq, Hkv, w_pre, w0)
+    ((1,), 2, 1, 1, 0),
+    ((100,), 4, 2, 40, 16),          # one partial tile, G = 3
+    ((128,), 4, 1, 64, 64),          # exactly one tile, G = 2
+    ((129,), 2, 2, 64, 1),           # tail tile of one row
+    ((300,), 8, 2, 100, 128),        # G = 3, tile-aligned window
+    ((777,), 4, 4, 160, 200),        # G = 5, window not tile-aligned
+    ((1500,), 4, 1, 512, 0),         # w0 = 0: every pair grouped
+    ((1024,), 4, 2, 256, 2000),      # window longer than the sequence
+    ((1024,), 4, 2, 4096, 64),       # G = 1
+    ((64, 0, 513, 1, 260), 8, 2, 128, 96),  # varlen with an empty sequence
+]
+
+
+@pytest.mark.parametrize("seqlens,Hq,Hkv,w_pre,w0", CASES)
+@pytest.mark.parametrize("kernel", ["tensor", "simt"])
+def test_bf16_cases_full(seqlens, Hq, Hkv, w_pre, w0, kernel):
+    J = jl()
+    q, k, v, cu = synth.random_case(sum(seqlens) + 7 * Hq + w0, seqlens, Hq, Hkv, 128, torch.bfloat16)
+    flags = J.JL_FLAG_SIMT if kernel == "simt" else 0
+    out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e6, flags=flags)
+    ro, rl = oracle.bifocal_attention(q, k, v, cu, w_pre, w0, 1e6)
+    assert_close(to_np(out), ro, torch.bfloat16, "out")
+    assert_close(to_np(lse), rl, torch.bfloat16, "lse")
+
+
+@pytest.mark.parametrize("seqlens,w_pre,w0", [((2048,), 4096, 300), ((700, 1300), 1300, 128)])
+def test_group_one_is_bitwise_plain_causal(seqlens, w_pre, w0):
+    # The pages: the base model is reproduced exactly inside its native context.
+    J = jl()
+    q, k, v, cu = synth.random_case(11, seqlens, 8, 2, 128, torch.bfloat16)
+    a, la = prefill_gpu(q, k, v, cu, w_pre, w0, 1e6)
+    b, lb = prefill_gpu(q, k, v, cu, w_pre, w0, 1e6, flags=J.JL_FLAG_PLAIN_CAUSAL)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_tensor_kernel_matches_simt_kernel():
+    J = jl()
+    q, k, v, cu = synth.random_case(5, (3000,), 8, 2, 128, torch.bfloat16)
+    a, la = prefill_gpu(q, k, v, cu, 1024, 333, 1e6)
+    b, lb = prefill_gpu(q, k, v, cu, 1024, 333, 1e6, flags=J.JL_FLAG_SIMT)
+    err = (a.float() - b.float()).abs()
+    assert err.max().item() < 2e-2 and err.mean().item() < 2e-3
+    ro, _ = oracle.bifocal_attention(q, k, v, cu, 1024, 333, 1e6, rows=np.arange(0, 3000, 97))
+    assert_close(to_np(a)[np.arange(0, 3000, 97)], ro, torch.bfloat16, "tensor vs oracle")
+
+
+def test_kernel_error_word_stays_clear():
+    J = jl()
+    q, k, v, cu = synth.random_case(3, (1000,), 4, 2, 128, torch.bfloat16)
+    dev = torch.device("cuda:0")
+    ws = torch.zeros(J.jl_bifocal_prefill_workspace_size(1, 1000, 4, 2, 128), dtype=torch.uint8, device=dev)
+    J.jl_bifocal_prefill(q.to(dev), k.to(dev), v.to(dev), cu.to(dev), 1000, 300, 200, 1e6, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+@pytest.mark.parametrize("name", ["prefill_32k_g1", "prefill_128k_g4", "varlen_4seq"])
+def test_full_size_workload_sampled_rows(name):
+    """Full-size workload in the benchmark's launch configuration; the oracle
+    evaluates a stratified sample of rows for every head."""
+    w = synth.WORKLOADS[name]
+    q, k, v, cu = synth.prefill_inputs(w)
+    out, lse = prefill_gpu(q, k, v, cu, w.w_pretrained, w.w0, w.rope_theta)
+    Gs = [oracle.group_size(L, w.w_pretrained) for L in w.seqlens]
+    rows = sample_rows(w.seqlens, w.w0, Gs, n_random=16 if len(w.seqlens) > 1 else 40)
+    ro, rl = oracle.bifocal_attention(q, k, v, cu, w.w_pretrained, w.w0, w.rope_theta, rows=rows)
+    got = to_np(out)[rows]
+    assert_close(got, ro, torch.bfloat16, name + " out")
+    assert_close(to_np(lse)[:, rows], rl, torch.bfloat16, name + " lse")
+    err = np.abs(got - ro)
+    # the relative L2 error is a sharper diagnostic than max-abs on small outputs
+    assert np.linalg.norm(got - ro) / np.linalg.norm(ro) < 1e-2
+    if max(Gs) > 1:
+        # discrimination: the grouped branch changes the result by much more
+        # than the kernel's error (a kernel that ignored grouping would fail)
+        po, _ = oracle.bifocal_attention(q, k, v, cu, w.w_pretrained, w.w0, w.rope_theta, rows=rows,
+                                         plain=True)
+        far = rows[np.isin(rows, rows)]
+        diff = np.abs(po - ro).mean()
+        assert diff > 5 * err.mean(), (diff, err.mean())

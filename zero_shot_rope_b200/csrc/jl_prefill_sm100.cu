@@ -1,0 +1,719 @@
+// Tensor-core prefill kernel for Dynamic Bifocal RoPE attention (sm_100a).
+//
+// Jet-Long technical summary, §2 "Mecanismos de Eficiência de Inferência":
+// the local window (base RoPE), the full causal pass over grouped queries and
+// keys, and the window pass over grouped queries and keys are merged by
+// inclusion–exclusion with LSE statistics, which gives the exact
+// distance-routed attention (§1 "Janela Local" / "Janela Remota").  This
+// kernel computes that exact value in one causal pass: every (query tile,
+// key tile) pair is visited with the base operands where all its distances
+// are < w0, with the grouped operands where all are >= w0, and twice (once
+// each, complementary masks) on the tile that straddles d = w0; one online
+// softmax runs over all visits.
+//
+// Per CTA: one 128-row query tile of one query head, head_dim 128.
+//   warps 0-3  softmax / correction / epilogue: thread r owns query row r and
+//              TMEM lane r; also rotates the query tile into grouped
+//              positions once (R(f(i) - i), §2 "Rotação de Correção").
+//   warp 4     TMA producer of Q and K tiles (128 x 128 bf16, SWIZZLE_128B).
+//   warp 5     TMEM allocator and the single-thread tcgen05.mma issuer:
+//              S = Q K^T (SS form) into a double-buffered TMEM S, then
+//              O += P V with P read from TMEM (TS form).
+//   warp 6     TMA producer of V tiles.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384) (fp32, lane = row);
+// P (bf16 pairs) overwrites the first 64 columns of its S buffer.
+//
+// The grouped keys K_g = R(f(j) - j) K~ are produced once per key by
+// prerotate_k_kernel; grouped visits load K_g tiles instead of K~ tiles.
+//
+// Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
+// records an error code, tells the other roles to stop, waits (bounded) for
+// its own copies and MMAs in flight, frees TMEM and returns.
+#include <cuda.h>
+
+#include "jl_common.cuh"
+
+namespace jl {
+namespace tc {
+
+constexpr int BM = 128;  // query rows per tile
+constexpr int BN = 128;  // keys per tile
+constexpr int HD = 128;  // head_dim
+constexpr int NKS = 2;   // K ring stages
+constexpr int NVS = 2;   // V ring stages
+constexpr int TILE_BYTES = BM * HD * 2;
+constexpr int HALF_BYTES = TILE_BYTES / 2;
+constexpr int NUM_THREADS = 224;
+constexpr int OFF_Q = 0;
+constexpr int OFF_QG = TILE_BYTES;
+constexpr int OFF_K = 2 * TILE_BYTES;
+constexpr int OFF_V = OFF_K + NKS * TILE_BYTES;
+constexpr int SMEM_TILES = OFF_V + NVS * TILE_BYTES;
+constexpr int SMEM_ALLOC = SMEM_TILES + 1024;  // slack to align the base to 1024 B
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_O = 256;
+constexpr int HI_INF = 1 << 30;
+
+// error codes (bit flags) written to the workspace error word
+constexpr int ERR_TIMEOUT_PRODUCER = 1;
+constexpr int ERR_TIMEOUT_MMA = 2;
+constexpr int ERR_TIMEOUT_SOFTMAX = 4;
+
+struct Params {
+  const int32_t *cu;
+  int batch, T, Hq, Hkv;
+  long long w_pre;
+  int w0, plain;
+  __nv_bfloat16 *out;
+  float *lse;
+  int *err;
+  float sl2;  // log2(e) / sqrt(D)
+};
+
+// ------------------------------------------------------------------ PTX glue
+__device__ __forceinline__ uint32_t su32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t gtime() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: false on timeout (records `code`) or when another role aborted.
+__device__ __noinline__ bool wait_b(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                    int *gerr, int code) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = gtime();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (gtime() - t0 > 2000000000ull) {
+        *abort_flag = 1;
+        if (gerr) atomicOr(gerr, code);
+        return false;
+      }
+    }
+  }
+}
+// Bounded wait used only to let this CTA's own copies / MMAs land before it
+// exits; ignores the abort flag.
+__device__ __noinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *gerr, int code) {
+  const uint64_t t0 = gtime();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try(bar, parity)) return;
+    if ((it & 31u) == 31u && gtime() - t0 > 2000000000ull) {
+      atomicOr(gerr, code);
+      return;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load(const CUtensorMap *map, uint64_t *bar, uint32_t dst, int c0,
+                                         int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(map), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   su32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+#define JL_R32(a) \
+  "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]), \
+  "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]),       \
+  "=r"(a[15]), "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]),     \
+  "=r"(a[22]), "=r"(a[23]), "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]),     \
+  "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
+#define JL_W32(a) \
+  "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]), "r"(a[8]), \
+  "r"(a[9]), "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15]), "r"(a[16]),    \
+  "r"(a[17]), "r"(a[18]), "r"(a[19]), "r"(a[20]), "r"(a[21]), "r"(a[22]), "r"(a[23]), "r"(a[24]),   \
+  "r"(a[25]), "r"(a[26]), "r"(a[27]), "r"(a[28]), "r"(a[29]), "r"(a[30]), "r"(a[31])
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : JL_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31, %32};" ::"r"(taddr),
+      JL_W32(r)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// wait::ld that also "redefines" the loaded registers, so no use of them can be
+// scheduled before the wait
+#define JL_RW32(a) \
+  "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]), \
+  "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]),       \
+  "+r"(a[15]), "+r"(a[16]), "+r"(a[17]), "+r"(a[18]), "+r"(a[19]), "+r"(a[20]), "+r"(a[21]),     \
+  "+r"(a[22]), "+r"(a[23]), "+r"(a[24]), "+r"(a[25]), "+r"(a[26]), "+r"(a[27]), "+r"(a[28]),     \
+  "+r"(a[29]), "+r"(a[30]), "+r"(a[31])
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : JL_RW32(r) : : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Shared-memory matrix descriptors (tcgen05 format, version 1).
+// K-major, 128-byte swizzle: 8-row atoms of 128 B, atoms 1024 B apart.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// MN-major, 128-byte swizzle: 64 contiguous N elements per 128 B row, 8 K rows
+// per 1024 B atom (SBO), N blocks of 64 `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, M = 128, N = 128.
+constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 16);  // B (= V) is MN-major
+
+// --------------------------------------------------------- tile schedule
+struct Tile {
+  int L, G, i0, i1, qt, bif;
+};
+
+// Visits of key tile kt: up to two (grouped part, base part).  For each,
+// columns c with (i - j0 - c) in [lo, hi] are kept when `mask` is set.
+struct Visit {
+  int grp, mask, lo, hi;
+};
+
+__device__ __forceinline__ int visits_of(const Tile &t, int w0, int kt, Visit (&vs)[2]) {
+  const int j0 = kt * BN;
+  const int j1 = min(j0 + BN - 1, t.L - 1);
+  const int dmin = t.i0 - j1, dmax = t.i1 - j0;
+  int n = 0;
+  if (!t.bif) {
+    vs[n++] = Visit{0, dmin < 0, 0, HI_INF};
+    return n;
+  }
+  if (dmax >= w0) vs[n++] = Visit{1, dmin < w0, w0, HI_INF};
+  if (w0 > 0 && dmin <= w0 - 1) vs[n++] = Visit{0, (dmin < 0) || (dmax > w0 - 1), 0, w0 - 1};
+  return n;
+}
+
+// ----------------------------------------------------------------- kernel
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                       const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
+                       const __grid_constant__ Params p, const __grid_constant__ InvFreq inv) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_q, bar_qg, bar_kf[NKS], bar_ke[NKS], bar_vf[NVS], bar_ve[NVS],
+      bar_sf[2], bar_pr[2], bar_od, bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item (uniform across the CTA; invalid items exit before any barrier)
+  const int s = blockIdx.z, h = blockIdx.y;
+  const int a = p.cu[s];
+  const int L = p.cu[s + 1] - a;
+  if (L <= 0 || a < 0 || a + L > p.T) return;
+  const int nqt = (L + BM - 1) / BM;
+  if ((int)blockIdx.x >= nqt) return;
+  Tile t;
+  t.L = L;
+  t.qt = nqt - 1 - (int)blockIdx.x;  // heaviest query tiles launch first
+  t.i0 = t.qt * BM;
+  t.i1 = min(t.i0 + BM - 1, L - 1);
+  t.G = p.plain ? 1 : (int)group_size(L, p.w_pre);
+  t.bif = t.G > 1;
+  const int kvh = h / (p.Hq / p.Hkv);
+  const bool need_qg = t.bif && t.i1 >= p.w0;
+
+  const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q, 1);
+    mbar_init(&bar_qg, 128);
+    for (int i = 0; i < NKS; ++i) { mbar_init(&bar_kf[i], 1); mbar_init(&bar_ke[i], 1); }
+    for (int i = 0; i < NVS; ++i) { mbar_init(&bar_vf[i], 1); mbar_init(&bar_ve[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&bar_sf[i], 1); mbar_init(&bar_pr[i], 128); }
+    mbar_init(&bar_od, 1);
+    mbar_init(&bar_drain, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (warp == 4 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mQ) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mK) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mV) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mKg) : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  const int tok_q0 = a + t.i0;
+  if (warp == 4) {
+    // ================= producer: Q, then K tiles in visit order =================
+    if (lane == 0) {
+      mbar_expect_tx(&bar_q, TILE_BYTES);
+      tma_load(&mQ, &bar_q, sbase + OFF_Q, 0, h, tok_q0);
+      tma_load(&mQ, &bar_q, sbase + OFF_Q + HALF_BYTES, 64, h, tok_q0);
+      int v = 0;
+      bool ok = true;
+      for (int kt = 0; kt <= t.qt && ok; ++kt) {
+        Visit vs[2];
+        const int nv = visits_of(t, p.w0, kt, vs);
+        for (int x = 0; x < nv; ++x, ++v) {
+          const int st = v % NKS;
+          if (v >= NKS && !(ok = wait_b(&bar_ke[st], ((v / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+            break;
+          const CUtensorMap *m = vs[x].grp ? &mKg : &mK;
+          const uint32_t dst = sbase + OFF_K + st * TILE_BYTES;
+          mbar_expect_tx(&bar_kf[st], TILE_BYTES);
+          tma_load(m, &bar_kf[st], dst, 0, kvh, a + kt * BN);
+          tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        }
+      }
+      // drain: every load issued must land before the CTA may exit
+      for (int u = max(0, v - NKS); u < v; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
+      wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
+    }
+  } else if (warp == 6) {
+    // ================= producer: V tiles in visit order =================
+    if (lane == 0) {
+      int v = 0;
+      bool ok = true;
+      for (int kt = 0; kt <= t.qt && ok; ++kt) {
+        Visit vs[2];
+        const int nv = visits_of(t, p.w0, kt, vs);
+        for (int x = 0; x < nv; ++x, ++v) {
+          const int st = v % NVS;
+          if (v >= NVS && !(ok = wait_b(&bar_ve[st], ((v / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+            break;
+          const uint32_t dst = sbase + OFF_V + st * TILE_BYTES;
+          mbar_expect_tx(&bar_vf[st], TILE_BYTES);
+          tma_load(&mV, &bar_vf[st], dst, 0, kvh, a + kt * BN);
+          tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        }
+      }
+      for (int u = max(0, v - NVS); u < v; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
+    }
+  } else if (warp == 5) {
+    // ================= MMA issuer (one thread) =================
+    if (lane == 0) {
+      bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
+      bool qg_seen = false;
+      int v = 0;
+      auto issue_pv = [&](int u) -> bool {
+        const int vs_ = u % NVS;
+        if (!wait_b(&bar_vf[vs_], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        if (!wait_b(&bar_pr[u & 1], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = sbase + OFF_V + vs_ * TILE_BYTES;
+        const uint32_t pcol = tmem + (uint32_t)((u & 1) * 128);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + COL_O, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV,
+                  (u > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bar_ve[vs_]);
+        umma_commit(&bar_od);
+        return true;
+      };
+      for (int kt = 0; kt <= t.qt && ok; ++kt) {
+        Visit vs[2];
+        const int nv = visits_of(t, p.w0, kt, vs);
+        for (int x = 0; x < nv && ok; ++x, ++v) {
+          if (vs[x].grp && !qg_seen) {
+            if (!(ok = wait_b(&bar_qg, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
+            qg_seen = true;
+          }
+          const int st = v % NKS;
+          if (!(ok = wait_b(&bar_kf[st], (v / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
+          tc_fence_after();
+          const uint32_t qaddr = sbase + (vs[x].grp ? OFF_QG : OFF_Q);
+          const uint32_t kaddr = sbase + OFF_K + st * TILE_BYTES;
+          const uint32_t scol = tmem + (uint32_t)((v & 1) * 128);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&bar_sf[v & 1]);
+          umma_commit(&bar_ke[st]);
+          if (v > 0 && !(ok = issue_pv(v - 1))) break;
+        }
+      }
+      if (ok && v > 0) issue_pv(v - 1);
+      // all MMAs issued so far must finish before TMEM is released
+      umma_commit(&bar_drain);
+      wait_drain(&bar_drain, 0, p.err, ERR_TIMEOUT_MMA);
+    }
+  } else {
+    // ================= softmax warpgroup (warps 0-3) =================
+    const int r = threadIdx.x;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int i = t.i0 + r;
+    bool ok = true;
+    if (need_qg) {
+      // rotate the query tile into grouped positions: Q_g = R(f(i) - i) Q~
+      ok = __all_sync(0xffffffffu, wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+      if (ok) {
+        for (int kk = 0; kk < 8; ++kk) {
+          const int u = r + 128 * kk;        // 16-byte chunk of the first half
+          const int row = u >> 3;
+          const int lc = (u & 7) ^ (row & 7);  // logical 8-column group
+          const int n = corr_n(min(t.i0 + row, L - 1), t.G);
+          uint4 xa = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + u * 16);
+          uint4 xb = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + HALF_BYTES + u * 16);
+          uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pa[e2]));
+            float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pb[e2]));
+            float c0, s0, c1, s1;
+            angle_cs(n, inv.v[lc * 8 + 2 * e2], c0, s0);
+            angle_cs(n, inv.v[lc * 8 + 2 * e2 + 1], c1, s1);
+            rot_back(fa.x, fb.x, c0, s0);
+            rot_back(fa.y, fb.y, c1, s1);
+            __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
+            __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
+            pa[e2] = *reinterpret_cast<uint32_t *>(&ra);
+            pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
+          }
+          *reinterpret_cast<uint4 *>(gbase + OFF_QG + u * 16) = xa;
+          *reinterpret_cast<uint4 *>(gbase + OFF_QG + HALF_BYTES + u * 16) = xb;
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bar_qg);
+    }
+
+    float m_run = -INFINITY, l_run = 0.f;
+    int v = 0;
+    for (int kt = 0; kt <= t.qt && ok; ++kt) {
+      Visit vs[2];
+      const int nv = visits_of(t, p.w0, kt, vs);
+      const int dc = i - kt * BN;  // column c has distance dc - c
+      for (int x = 0; x < nv && ok; ++x, ++v) {
+        const int b = v & 1;
+        ok = __all_sync(0xffffffffu, wait_b(&bar_sf[b], (v >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t scol = tmem + lane_base + (uint32_t)(b * 128);
+        float sv[128];
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(scol + 0, r0);
+          tmem_ld32(scol + 32, r1);
+          tmem_ld32(scol + 64, r2);
+          tmem_ld32(scol + 96, r3);
+          tmem_wait_ld_regs(r0);
+          tmem_wait_ld_regs(r1);
+          tmem_wait_ld_regs(r2);
+          tmem_wait_ld_regs(r3);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            sv[e] = __uint_as_float(r0[e]);
+            sv[32 + e] = __uint_as_float(r1[e]);
+            sv[64 + e] = __uint_as_float(r2[e]);
+            sv[96 + e] = __uint_as_float(r3[e]);
+          }
+        }
+        if (vs[x].mask) {
+          const int cmin = max(0, dc - vs[x].hi);
+          const int cmax = min(BN - 1, dc - vs[x].lo);
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < cmin || c > cmax) sv[c] = -INFINITY;
+        }
+        float mt = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) mt = fmaxf(mt, sv[c]);
+        mt *= p.sl2;
+        const float m_new = fmaxf(m_run, mt);
+        const bool need = (m_run != -INFINITY) && (m_new > m_run + 8.0f);
+        if (m_run == -INFINITY) m_run = m_new;
+        if (__any_sync(0xffffffffu, need)) {
+          // O holds PV of visits < v; PV_{v-1} may still run: wait for it
+          ok = __all_sync(0xffffffffu, wait_b(&bar_od, (v - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+          if (!ok) break;
+          tc_fence_after();
+          const float f = need ? ex2(m_run - m_new) : 1.0f;
+          if (need) {
+            l_run *= f;
+            m_run = m_new;
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t rr[32];
+            tmem_ld32(tmem + lane_base + COL_O + c4 * 32, rr);
+            tmem_wait_ld_regs(rr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
+            tmem_st32(tmem + lane_base + COL_O + c4 * 32, rr);
+          }
+          tmem_wait_st();
+        }
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        float lsum = 0.f;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float p0 = ex2(fmaf(sv[h2 * 64 + 2 * e], p.sl2, -m_use));
+            const float p1 = ex2(fmaf(sv[h2 * 64 + 2 * e + 1], p.sl2, -m_use));
+            lsum += p0 + p1;
+            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<uint32_t *>(&pb);
+          }
+          tmem_st32(scol + h2 * 32, pk);
+        }
+        l_run += lsum;
+        tmem_wait_st();
+        // the last visit: make sure PV_{v-1} is done so that exactly one PV
+        // (this visit's) is outstanding when the epilogue waits
+        const bool last = (kt == t.qt) && (x == nv - 1);
+        if (last && v > 0) {
+          ok = __all_sync(0xffffffffu, wait_b(&bar_od, (v - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+        }
+        tc_fence_before();
+        mbar_arrive(&bar_pr[b]);
+      }
+    }
+    // ---- epilogue: O / l -> bf16, LSE
+    if (ok && v > 0) ok = __all_sync(0xffffffffu, wait_b(&bar_od, (v - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      const bool row_ok = i < L;
+      __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * HD;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t rr[32];
+        tmem_ld32(tmem + lane_base + COL_O + c4 * 32, rr);
+        tmem_wait_ld_regs(rr);
+        if (row_ok) {
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+            uint4 o4;
+            uint32_t *po = reinterpret_cast<uint32_t *>(&o4);
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              __nv_bfloat162 ob = __floats2bfloat162_rn(__uint_as_float(rr[e8 * 8 + 2 * e2]) * inv_l,
+                                                        __uint_as_float(rr[e8 * 8 + 2 * e2 + 1]) * inv_l);
+              po[e2] = *reinterpret_cast<uint32_t *>(&ob);
+            }
+            *reinterpret_cast<uint4 *>(orow + c4 * 32 + e8 * 8) = o4;
+          }
+        }
+      }
+      if (row_ok && p.lse != nullptr)
+        p.lse[(size_t)h * p.T + tok_q0 + r] =
+            (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  // ---- teardown: every role has drained its own asynchronous work
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+// Grouped keys K_g = R(f(j) - j) K~ for every token of sequences with G > 1,
+// written once per key (all kv heads of a token share the angles).
+__global__ void __launch_bounds__(256)
+prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kg,
+                   const int32_t *__restrict__ cu, int batch, int T, int Hkv, long long w_pre,
+                   const __grid_constant__ InvFreq inv) {
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= (long long)T * 8) return;
+  const int tok = (int)(gid >> 3), cg = (int)(gid & 7);  // 8 pairs: k = 8cg .. 8cg+7
+  int lo = 0, hi = batch;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu[mid] <= tok) lo = mid; else hi = mid;
+  }
+  const int a = cu[lo], L = cu[lo + 1] - a, pos = tok - a;
+  if (L <= 0 || pos < 0 || pos >= L) return;
+  const int G = (int)group_size(L, w_pre);
+  if (G <= 1) return;  // never read: sequences with G = 1 have no grouped visit
+  const int n = corr_n(pos, G);
+  float cs[8], sn[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) angle_cs(n, inv.v[cg * 8 + e], cs[e], sn[e]);
+  for (int hh = 0; hh < Hkv; ++hh) {
+    const size_t base = ((size_t)tok * Hkv + hh) * HD + cg * 8;
+    uint4 xa = *reinterpret_cast<const uint4 *>(k + base);
+    uint4 xb = *reinterpret_cast<const uint4 *>(k + base + HD / 2);
+    uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pa[e2]));
+      float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pb[e2]));
+      rot_back(fa.x, fb.x, cs[2 * e2], sn[2 * e2]);
+      rot_back(fa.y, fb.y, cs[2 * e2 + 1], sn[2 * e2 + 1]);
+      __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
+      __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
+      pa[e2] = *reinterpret_cast<uint32_t *>(&ra);
+      pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
+    }
+    *reinterpret_cast<uint4 *>(kg + base) = xa;
+    *reinterpret_cast<uint4 *>(kg + base + HD / 2) = xb;
+  }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------ host
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [T, H, 128] bf16 viewed as a 3-D tensor (d, head, token); box 64 x 1 x 128.
+bool make_map(CUtensorMap *m, const void *base, int T, int H) {
+  EncodeTiledFn enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)tc::HD, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)tc::HD * 2, (cuuint64_t)H * tc::HD * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)tc::BM};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags) {
+  (void)batch; (void)Hq; (void)D; (void)flags;
+  return 256 + a256((size_t)T_total * Hkv * tc::HD * 2);
+}
+
+cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
+                              const int32_t *cu, int batch, int T_total, int max_seqlen, int Hq, int Hkv,
+                              long long w_pre, int w0, const InvFreq &inv, int plain, uint32_t flags,
+                              void *ws, size_t ws_bytes, cudaStream_t st, const char **why) {
+  (void)flags; (void)ws_bytes;
+  int *err = reinterpret_cast<int *>(ws);
+  __nv_bfloat16 *kg = reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(ws) + 256);
+  CUtensorMap mQ, mK, mV, mKg;
+  if (!make_map(&mQ, q, T_total, Hq) || !make_map(&mK, k, T_total, Hkv) || !make_map(&mV, v, T_total, Hkv) ||
+      !make_map(&mKg, kg, T_total, Hkv)) {
+    *why = "cuTensorMapEncodeTiled failed";
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  if (!plain) {
+    const long long n = (long long)T_total * 8;
+    tc::prerotate_k_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
+        (const __nv_bfloat16 *)k, kg, cu, batch, T_total, Hkv, w_pre, inv);
+    if ((e = cudaGetLastError()) != cudaSuccess) {
+      *why = "pre-rotation launch";
+      return e;
+    }
+  }
+  e = cudaFuncSetAttribute(tc::bifocal_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           tc::SMEM_ALLOC);
+  if (e != cudaSuccess) {
+    *why = "smem attribute";
+    return e;
+  }
+  tc::Params p;
+  p.cu = cu;
+  p.batch = batch;
+  p.T = T_total;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.w_pre = w_pre;
+  p.w0 = w0;
+  p.plain = plain;
+  p.out = (__nv_bfloat16 *)out;
+  p.lse = lse;
+  p.err = err;
+  p.sl2 = 1.4426950408889634f / sqrtf((float)tc::HD);
+  dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq, batch);
+  tc::bifocal_prefill_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) *why = "tensor-core prefill launch";
+  return e;
+}
+
+}  // namespace jl
