@@ -1,356 +1,361 @@
-// Split-KV decode kernel for Dynamic Bifocal RoPE attention.
+// Split-KV decode kernel for Dynamic Bifocal RoPE attention (sm_100a).
 //
-// One generation step: the new query (standard RoPE at position L-1) attends
-// to a standard-RoPE KV cache that is never rewritten.  Remote keys
-// (L-1 - j >= w0) are re-phased on the fly into grouped positions with the
-// correction rotation R(f(j) - j), the query with R(f(L-1) - (L-1))
-// (Jet-Long technical summary, §2 "Rotação de Correção On-the-Fly"); local
-// keys keep the base RoPE (§1 "Janela Local").  G is recomputed from L on the
-// device at every step.
+// One generation step: the new query (standard RoPE at position i = L-1)
+// attends to a standard-RoPE KV cache that is never rewritten.  Local keys
+// (i - j < w0) keep the base RoPE (Jet-Long technical summary, §1 "Janela
+// Local"); remote keys are scored at grouped positions through the correction
+// rotation of §2 "Rotação de Correção On-the-Fly".  Because RoPE rotations
+// compose additively,
+//     <R(delta_i) q~, R(delta_j) k~_j> = <q~, R(delta_j - delta_i) k~_j>,
+// so the kernel rotates each remote key once by the relative shift
+// delta_j - delta_i = -(n_j - n_i), n(p) = p - f(p), and dots it with the
+// stored query.  G is recomputed from L on the device at every step.
 //
-// Work split: CTA (split, kv head, sequence) owns keys [split*chunk, ...).
-//  pass 1  streams K rows with coalesced 8-byte loads: a key row of D bf16 is
-//          read by D/8 threads, thread t holding elements [4t, 4t+4) and
-//          [D/2 + 4t, D/2 + 4t + 4) so that each rotation pair (x_k, x_{k+D/2})
-//          lives in one thread.  The rotation angle n(j) * w_k with
-//          n(j) = j - f(j) advances by one position or none from key to key,
-//          so each thread carries cos/sin of its four angles as an fp32
-//          recurrence seeded exactly (fp64) at the start of its key range.
-//          The GQA group's scores are reduced across the row's threads with a
-//          transposed butterfly and kept in shared memory.
-//  pass 2  takes the per-head max, exponentiates in shared memory and
-//          streams V rows the same way, accumulating O per head.
-//  combine merges the splits with their (max, sum) statistics (the LSE merge).
+// CTA (split, kv head, sequence), 256 threads, keys [split*chunk, ...):
+//  * K and V tiles of 64 keys arrive by TMA (cp.async.bulk.tensor) in a
+//    3-stage shared-memory ring; thread 0 refills a stage once all eight
+//    warps have released it (mbarrier with one arrival per warp).
+//  * a key row of D elements is read by D/8 threads ("slot"): thread t holds
+//    elements [4t, 4t+4) and [D/2+4t, D/2+4t+4), i.e. whole rotation pairs.
+//    Slot s takes rows s, s+S, s+2S, ... (S = number of slots), so the
+//    rotation angle advances by a fixed stride; each thread carries the
+//    cos/sin of its four angles as an fp32 recurrence seeded in fp64.
+//  * per slot, an online softmax (running max / sum per GQA head) over its
+//    rows; the slots are merged at the end, the splits by a second kernel
+//    (the LSE merge of §2 "Mesclagem ... Inclusão–Exclusão" applied to key
+//    ranges).
 #include "jl_common.cuh"
+#include "jl_ptx.cuh"
 
 namespace jl {
 
-constexpr int DEC_THREADS = 128;
-constexpr int DEC_UNROLL = 4;
+constexpr int DEC_THREADS = 256;
+constexpr int DEC_TK = 64;  // keys per tile
+constexpr int DEC_NST = 3;  // ring stages (each: K tile + V tile)
 constexpr float LOG2E = 1.4426950408889634f;
-
-__device__ __forceinline__ void unpack4(uint2 u, float *x) {
-  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&u.x);
-  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&u.y);
-  float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
-  x[0] = fa.x; x[1] = fa.y; x[2] = fb.x; x[3] = fb.y;
-}
-
-__device__ __forceinline__ uint2 ld_stream8(const void *p) {
-  uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-               : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
+constexpr int DEC_ERR_TIMEOUT = 8;
 
 template <typename T>
-struct Row4;  // four consecutive elements of a row
+struct Row4;  // four consecutive row elements from shared memory, as fp32
 template <>
 struct Row4<__nv_bfloat16> {
-  static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float *x) { unpack4(ld_stream8(p), x); }
+  static __device__ __forceinline__ void load(const uint8_t *p, float *x) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  }
 };
 template <>
 struct Row4<float> {
-  static __device__ __forceinline__ void load(const float *p, float *x) {
-    float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+  static __device__ __forceinline__ void load(const uint8_t *p, float *x) {
+    const float4 v = *reinterpret_cast<const float4 *>(p);
     x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
   }
 };
 
-// Sum of GS per-head partials over the TPR threads of one key row.  On return
-// `out` is the full score of head `head` (valid in threads whose lowest
-// bits are zero, see `owner`).
+template <typename T>
+__device__ __forceinline__ void load_q4(const T *p, float *x);
+template <>
+__device__ __forceinline__ void load_q4<__nv_bfloat16>(const __nv_bfloat16 *p, float *x) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void load_q4<float>(const float *p, float *x) {
+  const float4 v = *reinterpret_cast<const float4 *>(p);
+  x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+}
+
+// Sum the GS per-head partials over the TPR threads of a slot and give every
+// thread of the slot all GS sums.
 template <int GS, int TPR>
-__device__ __forceinline__ void reduce_heads(const float (&v)[GS], int t, float &out, int &head,
-                                             bool &owner) {
+__device__ __forceinline__ void slot_allreduce(float (&v)[GS]) {
   if constexpr (GS == 4 && TPR >= 4) {
+    // transposed butterfly: two halving exchanges, then a plain reduction,
+    // then a broadcast of the four head sums
+    const int t = threadIdx.x % TPR;
     const bool hi = t & (TPR / 2);
-    float s0 = hi ? v[0] : v[2], s1 = hi ? v[1] : v[3];
+    const float s0 = hi ? v[0] : v[2], s1 = hi ? v[1] : v[3];
     float k0 = hi ? v[2] : v[0], k1 = hi ? v[3] : v[1];
     k0 += __shfl_xor_sync(0xffffffffu, s0, TPR / 2);
     k1 += __shfl_xor_sync(0xffffffffu, s1, TPR / 2);
     const bool hi2 = t & (TPR / 4);
-    float s = hi2 ? k0 : k1;
+    const float s = hi2 ? k0 : k1;
     float kk = hi2 ? k1 : k0;
     kk += __shfl_xor_sync(0xffffffffu, s, TPR / 4);
 #pragma unroll
     for (int o = TPR / 8; o >= 1; o >>= 1) kk += __shfl_xor_sync(0xffffffffu, kk, o);
-    out = kk;
-    head = 2 * (hi ? 1 : 0) + (hi2 ? 1 : 0);
-    owner = (t & (TPR / 4 - 1)) == 0;
-  } else {
-    float acc[GS];
+    // thread t now holds head 2*hi + hi2; fetch every head from its owner
+    const int base = (threadIdx.x & 31) & ~(TPR - 1);
 #pragma unroll
-    for (int g = 0; g < GS; ++g) {
-      acc[g] = v[g];
-#pragma unroll
-      for (int o = TPR / 2; o >= 1; o >>= 1) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], o);
+    for (int g = 0; g < 4; ++g) {
+      const int src = base + (g >> 1) * (TPR / 2) + (g & 1) * (TPR / 4);
+      v[g] = __shfl_sync(0xffffffffu, kk, src);
     }
-    // thread t < GS reports head t
-    out = acc[0];
+  } else {
 #pragma unroll
-    for (int g = 1; g < GS; ++g)
-      if (t == g) out = acc[g];
-    head = t;
-    owner = t < GS;
+    for (int g = 0; g < GS; ++g)
+#pragma unroll
+      for (int o = TPR / 2; o >= 1; o >>= 1) v[g] += __shfl_xor_sync(0xffffffffu, v[g], o);
   }
 }
 
+struct DecodeArgs {
+  const void *q;
+  const int32_t *seqlens;
+  int Lcap, Hq, Hkv;
+  long long w_pre;
+  int w0, plain, chunk, nsplit;
+  float *part_o, *part_ml;
+  int *err;
+};
+
 template <typename T, int D, int GS>
-__global__ void __launch_bounds__(DEC_THREADS)
-decode_partial_kernel(const T *__restrict__ q, const T *__restrict__ kc, const T *__restrict__ vc,
-                      const int32_t *__restrict__ seqlens, int Lcap, int Hq, int Hkv,
-                      long long w_pre, int w0, InvFreq inv, int plain, int chunk, int nsplit,
-                      float *__restrict__ part_o, float *__restrict__ part_ml) {
-  constexpr int TPR = D / 8;                 // threads per key row
-  constexpr int SLOTS = DEC_THREADS / TPR;   // key rows in flight per step
+__global__ void __launch_bounds__(DEC_THREADS, (GS <= 4 && sizeof(T) == 2) ? 2 : 1)
+decode_partial_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+                      const __grid_constant__ DecodeArgs p, const __grid_constant__ InvFreq inv) {
+  constexpr int TPR = D / 8;
+  constexpr int SLOTS = DEC_THREADS / TPR;
+  constexpr int RPS = DEC_TK / SLOTS;  // rows per slot per tile
   constexpr int HALF = D / 2;
-  extern __shared__ float smem[];            // scores [chunk][GS]; later the O reduction
-  __shared__ float head_m[GS], head_l[GS];
-  __shared__ float warp_red[DEC_THREADS / 32][GS];
+  constexpr int ROWB = D * (int)sizeof(T);
+  constexpr int TILEB = DEC_TK * ROWB;
+  constexpr int STAGEB = 2 * TILEB;
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[DEC_NST], empty[DEC_NST];
+  __shared__ volatile int abort_flag;
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, slot = tid / TPR, t = tid % TPR;
-  int L = seqlens[b];
+  int L = p.seqlens[b];
   // a length outside [0, min(Lcap, nsplit * chunk)] attends to nothing rather
   // than reading past the cache
-  if (L < 0 || L > Lcap || L > nsplit * chunk) L = 0;
-  const int kb = split * chunk;
-  const int ke = min(L, kb + chunk);
+  if (L < 0 || L > p.Lcap || L > p.nsplit * p.chunk) L = 0;
+  const int kb = split * p.chunk;
+  const int ke = min(L, kb + p.chunk);
   const int n = max(0, ke - kb);
-  const size_t pidx = ((size_t)b * Hq + (size_t)kvh * GS) * nsplit + split;  // head g adds g*nsplit
+  const size_t pidx = ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;  // + g * nsplit
 
   if (n == 0) {  // nothing to attend in this split
-    for (int idx = tid; idx < GS * D; idx += DEC_THREADS) {
-      const int g = idx / D, e = idx % D;
-      part_o[(pidx + (size_t)g * nsplit) * D + e] = 0.f;
-    }
+    for (int idx = tid; idx < GS * D; idx += DEC_THREADS)
+      p.part_o[(pidx + (size_t)(idx / D) * p.nsplit) * D + idx % D] = 0.f;
     if (tid < GS) {
-      part_ml[(pidx + (size_t)tid * nsplit) * 2 + 0] = -INFINITY;
-      part_ml[(pidx + (size_t)tid * nsplit) * 2 + 1] = 0.f;
+      p.part_ml[(pidx + (size_t)tid * p.nsplit) * 2 + 0] = -INFINITY;
+      p.part_ml[(pidx + (size_t)tid * p.nsplit) * 2 + 1] = 0.f;
     }
     return;
   }
+  const int ntiles = (n + DEC_TK - 1) / DEC_TK;
+  const int row0 = b * p.Lcap + kb;  // cache row of this split's first key
+  const uint32_t sbase = su32(smem);
 
-  const int i = L - 1;                                   // query position
-  const int G = plain ? 1 : (int)group_size(L, w_pre);
+  if (tid == 0) {
+    for (int s = 0; s < DEC_NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], DEC_THREADS / 32);
+    }
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  int issued = 0;  // tiles whose loads thread 0 has issued
+  if (tid == 0) {
+    for (int u = 0; u < min(DEC_NST, ntiles); ++u, ++issued) {
+      mbar_expect_tx(&full[u], STAGEB);
+      tma_load(&mK, &full[u], sbase + u * STAGEB, 0, kvh, row0 + u * DEC_TK);
+      tma_load(&mV, &full[u], sbase + u * STAGEB + TILEB, 0, kvh, row0 + u * DEC_TK);
+    }
+  }
+
+  const int i = L - 1;  // query position
+  const int G = p.plain ? 1 : (int)group_size(L, p.w_pre);
   const bool bif = G > 1;
-  const int j_local = (int)max(0LL, (long long)L - (long long)w0);  // keys >= j_local are local
-  const float sc = rsqrtf((float)D) * LOG2E;             // scores kept in log2 units
+  const int j_local = (int)max(0LL, (long long)L - (long long)p.w0);  // keys >= j_local are local
+  const float sl2 = rsqrtf((float)D) * LOG2E;
 
-  // ---- query: base and corrected copies of this thread's 8 elements per head
-  float qs[GS][8], qg[GS][8];
+  float qv[GS][8];
 #pragma unroll
   for (int g = 0; g < GS; ++g) {
-    const T *qp = q + ((size_t)b * Hq + (size_t)kvh * GS + g) * D;
-    Row4<T>::load(qp + 4 * t, &qs[g][0]);
-    Row4<T>::load(qp + HALF + 4 * t, &qs[g][4]);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) qg[g][e] = qs[g][e];
+    const T *qp = reinterpret_cast<const T *>(p.q) + ((size_t)b * p.Hq + (size_t)kvh * GS + g) * D;
+    load_q4<T>(qp + 4 * t, &qv[g][0]);
+    load_q4<T>(qp + HALF + 4 * t, &qv[g][4]);
   }
-  if (bif && i - 0 >= w0) {
+
+  // rotation state for this slot's current key j: cos/sin((n_j - n_i) w_k),
+  // advanced by SLOTS positions per row
+  float ec[4], es[4], w1c[4], w1s[4], w0c[4], w0s[4];
+  int rm = 0;
+  const int stride_full = SLOTS - SLOTS / max(G, 1);  // n advance without a carry
+  const int smod = SLOTS % max(G, 1);
+  if (bif) {
+    const int jf = kb + slot;
     const int ni = corr_n(i, G);
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      float c, s;
-      angle_cs(ni, inv.v[4 * t + p], c, s);
-#pragma unroll
-      for (int g = 0; g < GS; ++g) rot_back(qg[g][p], qg[g][4 + p], c, s);
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const double w = inv.v[4 * t + q4];
+      angle_cs(corr_n(jf, G) - ni, w, ec[q4], es[q4]);
+      angle_cs(stride_full, w, w1c[q4], w1s[q4]);
+      angle_cs(stride_full - 1, w, w0c[q4], w0s[q4]);
     }
+    rm = jf % G;
   }
 
-  // ---- per-slot contiguous key range, identical trip count for all slots
-  const int per = (n + SLOTS - 1) / SLOTS;
-  const int per_u = (per + DEC_UNROLL - 1) / DEC_UNROLL * DEC_UNROLL;
-  const int js = kb + slot * per;
-  const int je = min(ke, js + per);
-
-  // rotation recurrence state: cos/sin(n(j) w_k) for the slot's current key j
-  float ec[4], es[4], wc[4], ws[4];
-  int cnt = 0;  // (j + 1) % G
-  if (bif) {
-    const int n0 = corr_n(max(js, 0), G);
+  float m_run[GS], l_run[GS], o[GS][8];
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      angle_cs(n0, inv.v[4 * t + p], ec[p], es[p]);
-      angle_cs(1, inv.v[4 * t + p], wc[p], ws[p]);
-    }
-    cnt = (js + 1) % G;
+  for (int g = 0; g < GS; ++g) {
+    m_run[g] = -INFINITY;
+    l_run[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
   }
 
-  const size_t row_stride = (size_t)Hkv * D;
-  const T *kbase = kc + ((size_t)b * Lcap) * row_stride + (size_t)kvh * D;
-  const T *vbase = vc + ((size_t)b * Lcap) * row_stride + (size_t)kvh * D;
-
-  // ---- pass 1: scores
-  for (int u0 = 0; u0 < per_u; u0 += DEC_UNROLL) {
-    float kx[DEC_UNROLL][8];
+  bool ok = true;
+  for (int u = 0; u < ntiles; ++u) {
+    const int st = u % DEC_NST;
+    ok = __all_sync(0xffffffffu, wait_b(&full[st], (u / DEC_NST) & 1, &abort_flag, p.err, DEC_ERR_TIMEOUT));
+    if (!ok) break;
+    const uint8_t *kt = smem + st * STAGEB;
+    const uint8_t *vt = kt + TILEB;
+    const int j0 = kb + u * DEC_TK;
+    float sc[RPS][GS];
 #pragma unroll
-    for (int u = 0; u < DEC_UNROLL; ++u) {
-      const int j = js + u0 + u;
-      if (j < je) {
-        const T *kp = kbase + (size_t)j * row_stride;
-        Row4<T>::load(kp + 4 * t, &kx[u][0]);
-        Row4<T>::load(kp + HALF + 4 * t, &kx[u][4]);
-      } else {
+    for (int m = 0; m < RPS; ++m) {
+      const int r = slot + m * SLOTS;
+      const int j = j0 + r;
+      float kx[8];
+      Row4<T>::load(kt + r * ROWB + 4 * t * (int)sizeof(T), &kx[0]);
+      Row4<T>::load(kt + r * ROWB + (HALF + 4 * t) * (int)sizeof(T), &kx[4]);
+      if (bif && j < j_local) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kx[u][e] = 0.f;
+        for (int q4 = 0; q4 < 4; ++q4) rot_back(kx[q4], kx[4 + q4], ec[q4], es[q4]);
+      }
+#pragma unroll
+      for (int g = 0; g < GS; ++g) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaf(qv[g][e], kx[e], a);
+        sc[m][g] = a;
+      }
+      slot_allreduce<GS, TPR>(sc[m]);
+      const bool valid = j < ke;
+#pragma unroll
+      for (int g = 0; g < GS; ++g) sc[m][g] = valid ? sc[m][g] * sl2 : -INFINITY;
+      if (bif) {  // advance j -> j + SLOTS: n grows by SLOTS - floor((j+SLOTS)/G) + floor(j/G)
+        rm += smod;
+        const bool carry = rm >= G;
+        if (carry) rm -= G;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float wc = carry ? w0c[q4] : w1c[q4];
+          const float ws = carry ? w0s[q4] : w1s[q4];
+          const float c2 = ec[q4] * wc - es[q4] * ws;
+          const float s2 = es[q4] * wc + ec[q4] * ws;
+          ec[q4] = c2;
+          es[q4] = s2;
+        }
+      }
+    }
+    // online softmax over this slot's rows of the tile
+#pragma unroll
+    for (int g = 0; g < GS; ++g) {
+      float mt = sc[0][g];
+#pragma unroll
+      for (int m = 1; m < RPS; ++m) mt = fmaxf(mt, sc[m][g]);
+      if (mt > m_run[g]) {
+        const float f = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - mt);
+        l_run[g] *= f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[g][e] *= f;
+        m_run[g] = mt;
       }
     }
 #pragma unroll
-    for (int u = 0; u < DEC_UNROLL; ++u) {
-      const int j = js + u0 + u;
-      const bool remote = bif && j < j_local;
-      float part[GS];
-      if (remote) {
+    for (int m = 0; m < RPS; ++m) {
+      const int r = slot + m * SLOTS;
+      float vx[8];
+      Row4<T>::load(vt + r * ROWB + 4 * t * (int)sizeof(T), &vx[0]);
+      Row4<T>::load(vt + r * ROWB + (HALF + 4 * t) * (int)sizeof(T), &vx[4]);
 #pragma unroll
-        for (int p = 0; p < 4; ++p) rot_back(kx[u][p], kx[u][4 + p], ec[p], es[p]);
+      for (int g = 0; g < GS; ++g) {
+        const float pr = (sc[m][g] == -INFINITY) ? 0.f : exp2f(sc[m][g] - m_run[g]);
+        l_run[g] += pr;
 #pragma unroll
-        for (int g = 0; g < GS; ++g) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a = fmaf(qg[g][e], kx[u][e], a);
-          part[g] = a;
-        }
+        for (int e = 0; e < 8; ++e) o[g][e] = fmaf(pr, vx[e], o[g][e]);
+      }
+    }
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(&empty[st]);
+    if (tid == 0 && u + DEC_NST < ntiles) {
+      // refill this stage once every warp has released it
+      if (!wait_b(&empty[st], (u / DEC_NST) & 1, &abort_flag, p.err, DEC_ERR_TIMEOUT)) {
+        ok = false;
       } else {
-#pragma unroll
-        for (int g = 0; g < GS; ++g) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) a = fmaf(qs[g][e], kx[u][e], a);
-          part[g] = a;
-        }
+        const int un = u + DEC_NST;
+        mbar_expect_tx(&full[st], STAGEB);
+        tma_load(&mK, &full[st], sbase + st * STAGEB, 0, kvh, row0 + un * DEC_TK);
+        tma_load(&mV, &full[st], sbase + st * STAGEB + TILEB, 0, kvh, row0 + un * DEC_TK);
+        ++issued;
       }
-      float sres;
-      int head;
-      bool owner;
-      reduce_heads<GS, TPR>(part, t, sres, head, owner);
-      if (owner && j < je) smem[(j - kb) * GS + head] = sres * sc;
-      if (bif) {  // advance n(j) -> n(j+1): +1 unless j+1 starts a new group
-        const bool step = cnt != 0;
-        cnt = (cnt + 1 == G) ? 0 : cnt + 1;
-        if (step) {
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const float c2 = ec[p] * wc[p] - es[p] * ws[p];
-            const float s2 = es[p] * wc[p] + ec[p] * ws[p];
-            ec[p] = c2;
-            es[p] = s2;
-          }
-        }
-      }
+    }
+  }
+  // every load issued must land before the shared memory is reused or freed
+  if (tid == 0) {
+    for (int u = max(0, issued - DEC_NST); u < issued; ++u) {
+      // the last load of each stage is tile u (those before it were consumed)
+      wait_drain(&full[u % DEC_NST], (u / DEC_NST) & 1, p.err, DEC_ERR_TIMEOUT);
     }
   }
   __syncthreads();
 
-  // ---- per-head max and exponentials over this split's scores
-  {
-    float mx[GS];
+  // ---- merge the slots: (m, l, O) per head -> this split's partial
+  float *red_o = reinterpret_cast<float *>(smem);          // [SLOTS][GS][D]
+  float *red_m = red_o + SLOTS * GS * D;                    // [SLOTS][GS]
+  float *red_l = red_m + SLOTS * GS;                        // [SLOTS][GS]
 #pragma unroll
-    for (int g = 0; g < GS; ++g) mx[g] = -INFINITY;
-    for (int r = tid; r < n; r += DEC_THREADS)
-#pragma unroll
-      for (int g = 0; g < GS; ++g) mx[g] = fmaxf(mx[g], smem[r * GS + g]);
-#pragma unroll
-    for (int g = 0; g < GS; ++g)
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], o));
-    if ((tid & 31) == 0)
-#pragma unroll
-      for (int g = 0; g < GS; ++g) warp_red[tid >> 5][g] = mx[g];
-    __syncthreads();
-    if (tid < GS) {
-      float m = warp_red[0][tid];
-      for (int w = 1; w < DEC_THREADS / 32; ++w) m = fmaxf(m, warp_red[w][tid]);
-      head_m[tid] = m;
-    }
-    __syncthreads();
-    float sm[GS];
-#pragma unroll
-    for (int g = 0; g < GS; ++g) sm[g] = 0.f;
-    for (int r = tid; r < n; r += DEC_THREADS)
-#pragma unroll
-      for (int g = 0; g < GS; ++g) {
-        const float p = exp2f(smem[r * GS + g] - head_m[g]);
-        smem[r * GS + g] = p;
-        sm[g] += p;
-      }
-#pragma unroll
-    for (int g = 0; g < GS; ++g)
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) sm[g] += __shfl_xor_sync(0xffffffffu, sm[g], o);
-    __syncthreads();
-    if ((tid & 31) == 0)
-#pragma unroll
-      for (int g = 0; g < GS; ++g) warp_red[tid >> 5][g] = sm[g];
-    __syncthreads();
-    if (tid < GS) {
-      float l = 0.f;
-      for (int w = 0; w < DEC_THREADS / 32; ++w) l += warp_red[w][tid];
-      head_l[tid] = l;
-    }
-    __syncthreads();
-  }
-
-  // ---- pass 2: O = sum_j p_j V_j per head
-  float o[GS][8];
-#pragma unroll
-  for (int g = 0; g < GS; ++g)
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[g][e] = 0.f;
-  for (int u0 = 0; u0 < per_u; u0 += DEC_UNROLL) {
-    float vx[DEC_UNROLL][8];
-#pragma unroll
-    for (int u = 0; u < DEC_UNROLL; ++u) {
-      const int j = js + u0 + u;
-      if (j < je) {
-        const T *vp = vbase + (size_t)j * row_stride;
-        Row4<T>::load(vp + 4 * t, &vx[u][0]);
-        Row4<T>::load(vp + HALF + 4 * t, &vx[u][4]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < DEC_UNROLL; ++u) {
-      const int j = js + u0 + u;
-      if (j < je) {
-#pragma unroll
-        for (int g = 0; g < GS; ++g) {
-          const float p = smem[(j - kb) * GS + g];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o[g][e] = fmaf(p, vx[u][e], o[g][e]);
-        }
-      }
-    }
-  }
-  __syncthreads();  // scores no longer needed: reuse smem for the slot reduction
-
-  float *red = smem;  // [SLOTS][GS][D]
-#pragma unroll
-  for (int g = 0; g < GS; ++g)
+  for (int g = 0; g < GS; ++g) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int d = (e < 4) ? (4 * t + e) : (HALF + 4 * t + e - 4);
-      red[(slot * GS + g) * D + d] = o[g][e];
+      red_o[(slot * GS + g) * D + d] = o[g][e];
     }
+    if (t == 0) {
+      red_m[slot * GS + g] = m_run[g];
+      red_l[slot * GS + g] = l_run[g];
+    }
+  }
   __syncthreads();
   for (int idx = tid; idx < GS * D; idx += DEC_THREADS) {
     const int g = idx / D, d = idx % D;
-    float a = 0.f;
-#pragma unroll 4
-    for (int s = 0; s < SLOTS; ++s) a += red[(s * GS + g) * D + d];
-    part_o[(pidx + (size_t)g * nsplit) * D + d] = a;
-  }
-  if (tid < GS) {
-    part_ml[(pidx + (size_t)tid * nsplit) * 2 + 0] = head_m[tid];
-    part_ml[(pidx + (size_t)tid * nsplit) * 2 + 1] = head_l[tid];
+    float M = -INFINITY;
+    for (int s = 0; s < SLOTS; ++s) M = fmaxf(M, red_m[s * GS + g]);
+    float acc = 0.f, lsum = 0.f;
+    if (M != -INFINITY && ok) {
+      for (int s = 0; s < SLOTS; ++s) {
+        const float ms = red_m[s * GS + g];
+        if (ms == -INFINITY) continue;
+        const float w = exp2f(ms - M);
+        acc = fmaf(w, red_o[(s * GS + g) * D + d], acc);
+        lsum = fmaf(w, red_l[s * GS + g], lsum);
+      }
+    } else {
+      M = -INFINITY;
+    }
+    p.part_o[(pidx + (size_t)g * p.nsplit) * D + d] = acc;
+    if (d == 0) {
+      p.part_ml[(pidx + (size_t)g * p.nsplit) * 2 + 0] = M;
+      p.part_ml[(pidx + (size_t)g * p.nsplit) * 2 + 1] = lsum;
+    }
   }
 }
 
 // LSE-weighted merge of the splits of one (sequence, query head).
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
-decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml,
-                      int nsplit, T *__restrict__ out, float *__restrict__ lse) {
+decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml, int nsplit,
+                      T *__restrict__ out, float *__restrict__ lse) {
   const int bh = blockIdx.x, d = threadIdx.x;
   const float *ml = part_ml + (size_t)bh * nsplit * 2;
   float M = -INFINITY;
@@ -370,7 +375,7 @@ decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict_
 }
 
 // ---------------------------------------------------------------------------
-// host launcher (called from jl_api.cu after validation)
+// host
 // ---------------------------------------------------------------------------
 
 struct DecodePlan {
@@ -379,72 +384,100 @@ struct DecodePlan {
   size_t smem_bytes;
 };
 
-// Split count: aim at 592 CTAs (148 SMs x 4 resident 128-thread CTAs), keep a
-// split at most 2048 keys and a multiple of 32 keys.
-DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen) {
+static size_t decode_smem(int elem, int D, int GS) {
+  const int tpr = D / 8, slots = DEC_THREADS / tpr;
+  const size_t ring = (size_t)DEC_NST * 2 * DEC_TK * D * elem;
+  const size_t red = (size_t)slots * GS * (D + 2) * sizeof(float);
+  return ring > red ? ring : red;
+}
+
+// Split count: one wave of CTAs (148 SMs x CTAs resident per SM), splits of at
+// least one 64-key tile, rounded to whole tiles.
+DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int elem) {
   DecodePlan p;
-  const int target = 148 * 4;
+  const int GS = Hq / Hkv;
+  const int per_sm = (GS <= 4 && elem == 2) ? 2 : 1;
+  const int target = 148 * per_sm;
   const int per_bh = max(1, batch * Hkv);
-  int ns = (target + per_bh - 1) / per_bh;
+  int ns = max(1, target / per_bh);
   const int maxL = max(1, max_seqlen);
   int chunk = (maxL + ns - 1) / ns;
-  chunk = (chunk + 31) / 32 * 32;
-  if (chunk > 2048) chunk = 2048;
+  chunk = (chunk + DEC_TK - 1) / DEC_TK * DEC_TK;
   ns = (maxL + chunk - 1) / chunk;
   p.nsplit = ns;
   p.chunk = chunk;
-  const int GS = Hq / Hkv;
-  const int slots = DEC_THREADS / (D / 8);
-  const size_t a = (size_t)chunk * GS * sizeof(float);
-  const size_t r = (size_t)slots * GS * D * sizeof(float);
-  p.smem_bytes = a > r ? a : r;
+  p.smem_bytes = decode_smem(elem, D, GS);
   return p;
 }
 
+static bool make_cache_map(CUtensorMap *m, const void *base, int rows, int Hkv, int D, int elem) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * elem, (cuuint64_t)Hkv * D * elem};
+  cuuint32_t box[3] = {(cuuint32_t)D, 1, (cuuint32_t)DEC_TK};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+             const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int GS>
-static cudaError_t launch_decode_t(const void *q, const void *kc, const void *vc, const int32_t *seqlens,
-                                   int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                                   const InvFreq &inv, int plain, const DecodePlan &p, float *part_o,
-                                   float *part_ml, void *out, float *lse, cudaStream_t st) {
+static cudaError_t launch_decode_t(const CUtensorMap &mK, const CUtensorMap &mV, const DecodeArgs &a,
+                                   const InvFreq &inv, int B, const DecodePlan &pl, void *out, float *lse,
+                                   cudaStream_t st) {
   auto kern = decode_partial_kernel<T, D, GS>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)p.smem_bytes);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem_bytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nsplit, Hkv, B);
-  kern<<<grid, DEC_THREADS, p.smem_bytes, st>>>(
-      (const T *)q, (const T *)kc, (const T *)vc, seqlens, Lcap, Hq, Hkv, w_pre, w0, inv, plain,
-      p.chunk, p.nsplit, part_o, part_ml);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  decode_combine_kernel<T, D><<<B * Hq, D, 0, st>>>(part_o, part_ml, p.nsplit, (T *)out, lse);
+  dim3 grid(pl.nsplit, a.Hkv, B);
+  kern<<<grid, DEC_THREADS, pl.smem_bytes, st>>>(mK, mV, a, inv);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  decode_combine_kernel<T, D><<<B * a.Hq, D, 0, st>>>(a.part_o, a.part_ml, pl.nsplit, (T *)out, lse);
   return cudaGetLastError();
 }
 
 template <typename T, int D>
-static cudaError_t launch_decode_d(int GS, const void *q, const void *kc, const void *vc,
-                                   const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv,
-                                   long long w_pre, int w0, const InvFreq &inv, int plain,
-                                   const DecodePlan &p, float *po, float *pml, void *out, float *lse,
+static cudaError_t launch_decode_d(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const DecodeArgs &a,
+                                   const InvFreq &inv, int B, const DecodePlan &pl, void *out, float *lse,
                                    cudaStream_t st) {
   switch (GS) {
-    case 1: return launch_decode_t<T, D, 1>(q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, po, pml, out, lse, st);
-    case 2: return launch_decode_t<T, D, 2>(q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, po, pml, out, lse, st);
-    case 4: return launch_decode_t<T, D, 4>(q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, po, pml, out, lse, st);
-    case 8: return launch_decode_t<T, D, 8>(q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, po, pml, out, lse, st);
+    case 1: return launch_decode_t<T, D, 1>(mK, mV, a, inv, B, pl, out, lse, st);
+    case 2: return launch_decode_t<T, D, 2>(mK, mV, a, inv, B, pl, out, lse, st);
+    case 4: return launch_decode_t<T, D, 4>(mK, mV, a, inv, B, pl, out, lse, st);
+    case 8: return launch_decode_t<T, D, 8>(mK, mV, a, inv, B, pl, out, lse, st);
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
-                          const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre,
-                          int w0, const InvFreq &inv, int plain, const DecodePlan &p, float *part_o,
-                          float *part_ml, void *out, float *lse, cudaStream_t st) {
+                          const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
+                          const InvFreq &inv, int plain, const DecodePlan &pl, float *part_o, float *part_ml,
+                          int *err, void *out, float *lse, cudaStream_t st) {
+  const int elem = bf16 ? 2 : 4;
+  CUtensorMap mK, mV;
+  if (!make_cache_map(&mK, kc, B * Lcap, Hkv, D, elem) || !make_cache_map(&mV, vc, B * Lcap, Hkv, D, elem))
+    return cudaErrorInvalidValue;
+  DecodeArgs a;
+  a.q = q;
+  a.seqlens = seqlens;
+  a.Lcap = Lcap;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.w_pre = w_pre;
+  a.w0 = w0;
+  a.plain = plain;
+  a.chunk = pl.chunk;
+  a.nsplit = pl.nsplit;
+  a.part_o = part_o;
+  a.part_ml = part_ml;
+  a.err = err;
   if (bf16) {
-    if (D == 128) return launch_decode_d<__nv_bfloat16, 128>(GS, q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, part_o, part_ml, out, lse, st);
-    if (D == 64) return launch_decode_d<__nv_bfloat16, 64>(GS, q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, part_o, part_ml, out, lse, st);
+    if (D == 128) return launch_decode_d<__nv_bfloat16, 128>(GS, mK, mV, a, inv, B, pl, out, lse, st);
+    if (D == 64) return launch_decode_d<__nv_bfloat16, 64>(GS, mK, mV, a, inv, B, pl, out, lse, st);
   } else {
-    if (D == 128) return launch_decode_d<float, 128>(GS, q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, part_o, part_ml, out, lse, st);
-    if (D == 64) return launch_decode_d<float, 64>(GS, q, kc, vc, seqlens, B, Lcap, Hq, Hkv, w_pre, w0, inv, plain, p, part_o, part_ml, out, lse, st);
+    if (D == 128) return launch_decode_d<float, 128>(GS, mK, mV, a, inv, B, pl, out, lse, st);
+    if (D == 64) return launch_decode_d<float, 64>(GS, mK, mV, a, inv, B, pl, out, lse, st);
   }
   return cudaErrorInvalidValue;
 }

@@ -32,6 +32,7 @@
 #include <cuda.h>
 
 #include "jl_common.cuh"
+#include "jl_ptx.cuh"
 
 namespace jl {
 namespace tc {
@@ -70,73 +71,6 @@ struct Params {
   float sl2;  // log2(e) / sqrt(D)
 };
 
-// ------------------------------------------------------------------ PTX glue
-__device__ __forceinline__ uint32_t su32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t n) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(su32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t gtime() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait: false on timeout (records `code`) or when another role aborted.
-__device__ __noinline__ bool wait_b(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                    int *gerr, int code) {
-  if (mbar_try(bar, parity)) return true;
-  const uint64_t t0 = gtime();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try(bar, parity)) return true;
-    if ((it & 31u) == 0) {
-      if (*abort_flag) return false;
-      if (gtime() - t0 > 2000000000ull) {
-        *abort_flag = 1;
-        if (gerr) atomicOr(gerr, code);
-        return false;
-      }
-    }
-  }
-}
-// Bounded wait used only to let this CTA's own copies / MMAs land before it
-// exits; ignores the abort flag.
-__device__ __noinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *gerr, int code) {
-  const uint64_t t0 = gtime();
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try(bar, parity)) return;
-    if ((it & 31u) == 31u && gtime() - t0 > 2000000000ull) {
-      atomicOr(gerr, code);
-      return;
-    }
-  }
-}
-__device__ __forceinline__ void tma_load(const CUtensorMap *map, uint64_t *bar, uint32_t dst, int c0,
-                                         int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(map), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
@@ -237,13 +171,16 @@ __device__ __forceinline__ int visits_of(const Tile &t, int w0, int kt, Visit (&
   const int j0 = kt * BN;
   const int j1 = min(j0 + BN - 1, t.L - 1);
   const int dmin = t.i0 - j1, dmax = t.i1 - j0;
+  // the diagonal tile always needs the causal mask: besides j > i it holds
+  // the keys at or past L (zero-filled or the next sequence's)
+  const int diag = kt == t.qt;
   int n = 0;
   if (!t.bif) {
-    vs[n++] = Visit{0, dmin < 0, 0, HI_INF};
+    vs[n++] = Visit{0, diag, 0, HI_INF};
     return n;
   }
-  if (dmax >= w0) vs[n++] = Visit{1, dmin < w0, w0, HI_INF};
-  if (w0 > 0 && dmin <= w0 - 1) vs[n++] = Visit{0, (dmin < 0) || (dmax > w0 - 1), 0, w0 - 1};
+  if (dmax >= w0) vs[n++] = Visit{1, diag || dmin < w0, w0, HI_INF};
+  if (w0 > 0 && dmin <= w0 - 1) vs[n++] = Visit{0, diag || dmax > w0 - 1, 0, w0 - 1};
   return n;
 }
 
@@ -627,25 +564,9 @@ prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restric
 // ------------------------------------------------------------------ host
 namespace {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
 // [T, H, 128] bf16 viewed as a 3-D tensor (d, head, token); box 64 x 1 x 128.
 bool make_map(CUtensorMap *m, const void *base, int T, int H) {
-  EncodeTiledFn enc = get_encode();
+  EncodeTiledFn enc = get_encode_tiled();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)tc::HD, (cuuint64_t)H, (cuuint64_t)T};
   cuuint64_t strides[2] = {(cuuint64_t)tc::HD * 2, (cuuint64_t)H * tc::HD * 2};
@@ -660,6 +581,18 @@ bool make_map(CUtensorMap *m, const void *base, int T, int H) {
 size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
 
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags) {
   (void)batch; (void)Hq; (void)D; (void)flags;

@@ -1,0 +1,84 @@
+// PTX helpers shared by the sm_100a kernels: mbarriers, bounded waits and
+// TMA tensor loads.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+namespace jl {
+
+__device__ __forceinline__ uint32_t su32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t n) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(n));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t *b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(su32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t gtime() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait: false on timeout (records `code`) or when another role aborted.
+static __device__ __noinline__ bool wait_b(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                    int *gerr, int code) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = gtime();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (gtime() - t0 > 2000000000ull) {
+        *abort_flag = 1;
+        if (gerr) atomicOr(gerr, code);
+        return false;
+      }
+    }
+  }
+}
+// Bounded wait used only to let this CTA's own copies / MMAs land before it
+// exits; ignores the abort flag.
+static __device__ __noinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *gerr, int code) {
+  const uint64_t t0 = gtime();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try(bar, parity)) return;
+    if ((it & 31u) == 31u && gtime() - t0 > 2000000000ull) {
+      atomicOr(gerr, code);
+      return;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load(const CUtensorMap *map, uint64_t *bar, uint32_t dst, int c0,
+                                         int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(map), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Host: cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+}  // namespace jl
