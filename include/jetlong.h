@@ -172,6 +172,43 @@ jl_status jl_bifocal_decode(const void *q, const void *k_cache,
                             void *workspace, size_t workspace_bytes,
                             jl_dtype dtype, uint32_t flags, void *stream);
 
+/*
+ * jl_bifocal_decode_noalloc — jl_bifocal_decode without a caller workspace.
+ * (An addition of this library for callers that cannot allocate; the paper
+ * has no counterpart.)
+ *
+ * Some callers cannot call cudaMalloc: a plugin hosted by a runtime that owns
+ * the whole device-memory budget, or a latency-critical generation loop that
+ * must not risk the implicit device synchronisation an allocation can bring.
+ * This entry point allocates nothing.  Its scratch (split-KV partial results
+ * and an error word) is a fixed array of JL_DECODE_NOALLOC_SCRATCH_BYTES in
+ * the library's device image, held by every GPU that loads the library until
+ * the process exits.
+ *
+ *   Arguments, layouts and results are those of jl_bifocal_decode, minus the
+ *   workspace.  A decode whose jl_bifocal_decode_workspace_size(...) exceeds
+ *   JL_DECODE_NOALLOC_SCRATCH_BYTES is rejected with JL_ERR_WORKSPACE before
+ *   any launch (jl_last_error() says how much it needed).
+ *   The first call on a device (with that device current) looks up the
+ *   array's device address once (cudaGetSymbolAddress); make that first call
+ *   before any stream capture.  A failed lookup returns JL_ERR_CUDA.
+ *   All calls share the one array, which keeps the last call's contents; the
+ *   kernels clear what must start at zero.  Calls that overlap on the GPU
+ *   (different streams, or different host threads, on the same device) race
+ *   on the array: serialise them.
+ */
+#define JL_DECODE_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+jl_status jl_bifocal_decode_noalloc(const void *q, const void *k_cache,
+                                    const void *v_cache,
+                                    const int32_t *seqlens, int32_t batch,
+                                    int32_t cache_capacity, int32_t max_seqlen,
+                                    int32_t n_q_heads, int32_t n_kv_heads,
+                                    int32_t head_dim, int64_t w_pretrained,
+                                    int32_t w0, double rope_theta, void *out,
+                                    float *lse, jl_dtype dtype, uint32_t flags,
+                                    void *stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif

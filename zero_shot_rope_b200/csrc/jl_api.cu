@@ -78,6 +78,16 @@ jl_status cuda_fail(cudaError_t e, const char *what) {
 
 }  // namespace
 
+namespace jl {
+// Record a message for jl_last_error() from other translation units.
+void set_last_error(const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+}  // namespace jl
+
 extern "C" {
 
 const char *jl_status_string(jl_status s) {

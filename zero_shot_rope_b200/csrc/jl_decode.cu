@@ -483,3 +483,79 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
 }
 
 }  // namespace jl
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode entry point
+//
+// Some callers cannot call cudaMalloc: a plugin hosted by a runtime that owns
+// the whole device-memory budget (its allocator hands out nothing outside its
+// own pools), or a latency-critical generation loop that must not risk the
+// implicit device synchronisation an allocation can cause.  For them
+// jl_bifocal_decode_noalloc runs the same split-KV decode with its scratch
+// (the per-split partial results and an error word) in a fixed array that
+// lives in the library's own device image.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+#include "../../include/jetlong.h"
+
+namespace jl {
+void set_last_error(const char *fmt, ...);
+}
+
+// File-scope scratch of JL_DECODE_NOALLOC_SCRATCH_BYTES.  Every GPU that loads
+// the library holds it until the process exits.  In host code this name is
+// only a host-side stand-in: the device address comes from
+// cudaGetSymbolAddress, taken once per device below.
+static __device__ __align__(256) uint8_t g_decode_scratch[JL_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_scratch_mu;
+void *g_scratch_addr[256] = {nullptr};
+
+// Device address of g_decode_scratch on the current device (set up on the
+// first call made with that device current).
+cudaError_t scratch_for_current_device(void **out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+extern "C" jl_status jl_bifocal_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                               const int32_t *seqlens, int32_t batch, int32_t cache_capacity,
+                                               int32_t max_seqlen, int32_t n_q_heads, int32_t n_kv_heads,
+                                               int32_t head_dim, int64_t w_pretrained, int32_t w0,
+                                               double rope_theta, void *out, float *lse, jl_dtype dtype,
+                                               uint32_t flags, void *stream) {
+  const size_t need = jl_bifocal_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen);
+  if (need > (size_t)JL_DECODE_NOALLOC_SCRATCH_BYTES) {
+    jl::set_last_error("this decode needs %zu bytes of scratch; the allocation-free entry point has a fixed %u "
+                       "bytes (use jl_bifocal_decode with a caller workspace)",
+                       need, (unsigned)JL_DECODE_NOALLOC_SCRATCH_BYTES);
+    return JL_ERR_WORKSPACE;
+  }
+  if (batch <= 0)  // nothing to do (or an argument error): no scratch needed
+    return jl_bifocal_decode(q, k_cache, v_cache, seqlens, batch, cache_capacity, max_seqlen, n_q_heads,
+                             n_kv_heads, head_dim, w_pretrained, w0, rope_theta, out, lse, nullptr, 0, dtype,
+                             flags, stream);
+  void *scratch = nullptr;
+  const cudaError_t e = scratch_for_current_device(&scratch);
+  if (e != cudaSuccess) {
+    jl::set_last_error("cudaGetSymbolAddress of the decode scratch failed: %s", cudaGetErrorString(e));
+    return JL_ERR_CUDA;
+  }
+  return jl_bifocal_decode(q, k_cache, v_cache, seqlens, batch, cache_capacity, max_seqlen, n_q_heads, n_kv_heads,
+                           head_dim, w_pretrained, w0, rope_theta, out, lse, scratch,
+                           (size_t)JL_DECODE_NOALLOC_SCRATCH_BYTES, dtype, flags, stream);
+}

@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_decode.restype = ctypes.c_int
     L.jl_bifocal_decode.argtypes = [c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64,
                                     c_i32, c_d, c_p, c_p, c_p, c_sz, ctypes.c_int, c_u32, c_p]
+    L.jl_bifocal_decode_noalloc.restype = ctypes.c_int
+    L.jl_bifocal_decode_noalloc.argtypes = [c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                            c_i64, c_i32, c_d, c_p, c_p, ctypes.c_int, c_u32, c_p]
     _lib = L
     return L
 
@@ -158,4 +161,22 @@ def jl_bifocal_decode(q, k_cache, v_cache, seqlens, max_seqlen, w_pretrained, w0
                                    float(rope_theta), _ptr(out), _ptr(lse), _ptr(ws),
                                    0 if ws is None else ws.numel() * ws.element_size(),
                                    _dtype_code(q), int(flags), _stream(stream)))
+    return out, lse
+
+
+JL_DECODE_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def jl_bifocal_decode_noalloc(q, k_cache, v_cache, seqlens, max_seqlen, w_pretrained, w0, rope_theta,
+                              out, lse=None, flags=0, stream=None):
+    """jl_bifocal_decode for callers that cannot allocate device memory: the
+    library supplies the scratch from a fixed array in its device image
+    (JL_DECODE_NOALLOC_SCRATCH_BYTES), so ``out`` must be given and nothing
+    is allocated.  Calls that overlap on the GPU share that array and race."""
+    B, Hq, D = q.shape
+    Lcap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _check(lib().jl_bifocal_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, Lcap,
+                                           int(max_seqlen), Hq, Hkv, D, int(w_pretrained), int(w0),
+                                           float(rope_theta), _ptr(out), _ptr(lse), _dtype_code(q), int(flags),
+                                           _stream(stream)))
     return out, lse
