@@ -74,12 +74,14 @@ def kernel_traffic(name):
         d = json.load(f).get(name)
     if not d:
         return None
-    src = os.path.join(ROOT, d["source"])
-    if not os.path.exists(src):
-        return None
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    return d["bytes_per_launch"] if sha == d["source_sha"] else None
+    h = hashlib.sha256()
+    for src in d["sources"]:
+        path = os.path.join(ROOT, src)
+        if not os.path.exists(path):
+            return None
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return d["bytes_per_launch"] if h.hexdigest()[:16] == d["source_sha"] else None
 
 
 class ClockSampler:
