@@ -89,3 +89,20 @@ def test_decode_zero_length_writes_zero():
     assert torch.all(out[0] == 0) and torch.all(torch.isinf(lse[0]))
     ro, _ = oracle.bifocal_decode(q[1:], kc[1:], vc[1:], [50], 16, 8, 1e4)
     assert_close(to_np(out[1:]), ro, torch.bfloat16, "row 1")
+
+
+@pytest.mark.parametrize("D,dtype", [(128, torch.bfloat16), (64, torch.bfloat16), (128, torch.float32)])
+def test_decode_ignores_garbage_past_the_length(D, dtype):
+    # cache rows at and past L may hold anything (here NaN): they must not
+    # reach the result (a 0 * NaN in the PV product would)
+    g = torch.Generator().manual_seed(17)
+    L, cap = 1000, 1200
+    q = torch.randn(1, 8, D, generator=g).to(dtype)
+    kc = torch.randn(1, cap, 2, D, generator=g).to(dtype)
+    vc = torch.randn(1, cap, 2, D, generator=g).to(dtype)
+    kc[:, L:] = float("nan")
+    vc[:, L:] = float("nan")
+    out, lse = decode_gpu(q, kc, vc, [L], cap, 300, 64, 1e6)
+    ro, rl = oracle.bifocal_decode(q, kc, vc, [L], 300, 64, 1e6)
+    assert_close(to_np(out), ro, dtype, "out")
+    assert_close(to_np(lse), rl, dtype, "lse")

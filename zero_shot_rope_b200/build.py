@@ -12,7 +12,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libjetlong.so")
-SOURCES = ["jl_api.cu", "jl_simt.cu", "jl_decode.cu", "jl_prefill_sm100.cu"]
+SOURCES = ["jl_api.cu", "jl_simt.cu", "jl_decode.cu", "jl_decode_sm100.cu", "jl_prefill_sm100.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -32,7 +32,8 @@ def nvcc() -> str:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
-    deps = srcs + [os.path.join(CSRC, "jl_common.cuh"), os.path.join(ROOT, "include", "jetlong.h")]
+    deps = srcs + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
+    deps.append(os.path.join(ROOT, "include", "jetlong.h"))
     if not force and os.path.exists(LIB):
         newest = max(os.path.getmtime(d) for d in deps)
         if os.path.getmtime(LIB) >= newest:

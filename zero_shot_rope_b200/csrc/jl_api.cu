@@ -18,10 +18,11 @@ struct DecodePlan {
   size_t smem_bytes;
 };
 DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int elem);
+size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen);
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
-                          const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                          const InvFreq &inv, int plain, const DecodePlan &pl, float *part_o, float *part_ml,
-                          int *err, void *out, float *lse, cudaStream_t st);
+                          const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
+                          long long w_pre, int w0, const InvFreq &inv, int plain, float *part_o,
+                          float *part_ml, int *err, void *out, float *lse, cudaStream_t st);
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags);
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
                               const int32_t *cu, int batch, int T_total, int max_seqlen, int Hq,
@@ -173,11 +174,9 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
 size_t jl_bifocal_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
                                         int32_t head_dim, int32_t max_seqlen) {
   if (batch <= 0 || n_q_heads <= 0 || n_kv_heads <= 0 || head_dim <= 0 || max_seqlen < 0) return 0;
-  // sized for the larger element type so that one buffer serves both dtypes
-  const jl::DecodePlan p2 = jl::decode_plan(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen, 2);
-  const jl::DecodePlan p4 = jl::decode_plan(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen, 4);
-  const size_t ns = (size_t)(p2.nsplit > p4.nsplit ? p2.nsplit : p4.nsplit);
-  const size_t rows = (size_t)batch * n_q_heads * ns;
+  if (n_q_heads % n_kv_heads != 0) return 0;
+  // one layout serves every dtype and both decode kernels
+  const size_t rows = jl::decode_partial_rows(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen);
   return 256 + align256(rows * head_dim * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
 
@@ -209,9 +208,7 @@ jl_status jl_bifocal_decode(const void *q, const void *k_cache, const void *v_ca
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(JL_ERR_WORKSPACE, "workspace must be 256-byte aligned");
 
-  const int elem = dtype == JL_BF16 ? 2 : 4;
-  const jl::DecodePlan p = jl::decode_plan(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen, elem);
-  const size_t rows = (size_t)batch * n_q_heads * p.nsplit;
+  const size_t rows = jl::decode_partial_rows(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen);
   int *err = (int *)workspace;
   float *part_o = (float *)((char *)workspace + 256);
   float *part_ml = (float *)((char *)workspace + 256 + align256(rows * head_dim * sizeof(float)));
@@ -220,8 +217,8 @@ jl_status jl_bifocal_decode(const void *q, const void *k_cache, const void *v_ca
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e == cudaSuccess)
     e = jl::launch_decode(dtype == JL_BF16, head_dim, gs, q, k_cache, v_cache, seqlens, batch, cache_capacity,
-                          n_q_heads, n_kv_heads, w_pretrained, w0, inv, (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0,
-                          p, part_o, part_ml, err, out, lse, st);
+                          max_seqlen, n_q_heads, n_kv_heads, w_pretrained, w0, inv,
+                          (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0, part_o, part_ml, err, out, lse, st);
   return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
 }
 

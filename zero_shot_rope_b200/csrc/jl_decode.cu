@@ -275,6 +275,7 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap mK, const __grid_const
 #pragma unroll
     for (int m = 0; m < RPS; ++m) {
       const int r = slot + m * SLOTS;
+      if (j0 + r >= ke) continue;  // past the last key: the cache may hold anything there
       float vx[8];
       Row4<T>::load(vt + r * ROWB + 4 * t * (int)sizeof(T), &vx[0]);
       Row4<T>::load(vt + r * ROWB + (HALF + 4 * t) * (int)sizeof(T), &vx[4]);
@@ -450,11 +451,60 @@ static cudaError_t launch_decode_d(int GS, const CUtensorMap &mK, const CUtensor
   return cudaErrorInvalidValue;
 }
 
+void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk);
+cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
+                             const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
+                             const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o, float *part_ml,
+                             int *err, cudaStream_t st);
+
+static bool use_tc_decode(bool bf16, int D, int GS) { return bf16 && D == 128 && GS <= 8; }
+
+// Rows of split partials the workspace must hold: the largest of the plans
+// either decode kernel may use.
+size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
+  const int GS = Hq / Hkv;
+  int ns = decode_plan(batch, Hq, Hkv, D, max_seqlen, 2).nsplit;
+  ns = max(ns, decode_plan(batch, Hq, Hkv, D, max_seqlen, 4).nsplit);
+  if (use_tc_decode(true, D, GS)) {
+    int nt, ct;
+    decode_tc_plan(batch, Hkv, max_seqlen, &nt, &ct);
+    ns = max(ns, nt);
+  }
+  return (size_t)batch * Hq * ns;
+}
+
+static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv) {
+  // bf16 cache viewed as (d, head, row); 64 x 1 x 128 boxes, 128-byte swizzle
+  EncodeTiledFn enc = get_encode_tiled();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)Hkv, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {256, (cuuint64_t)Hkv * 256};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
-                          const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                          const InvFreq &inv, int plain, const DecodePlan &pl, float *part_o, float *part_ml,
-                          int *err, void *out, float *lse, cudaStream_t st) {
+                          const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
+                          long long w_pre, int w0, const InvFreq &inv, int plain, float *part_o,
+                          float *part_ml, int *err, void *out, float *lse, cudaStream_t st) {
   const int elem = bf16 ? 2 : 4;
+  if (use_tc_decode(bf16, D, GS)) {
+    CUtensorMap tK, tV;
+    if (!make_tile_map(&tK, kc, B * Lcap, Hkv) || !make_tile_map(&tV, vc, B * Lcap, Hkv))
+      return cudaErrorInvalidValue;
+    int ns, chunk;
+    decode_tc_plan(B, Hkv, max_seqlen, &ns, &chunk);
+    cudaError_t e = launch_decode_tc(GS, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, Hq, Hkv, w_pre, w0,
+                                     inv, plain, ns, chunk, part_o, part_ml, err, st);
+    if (e != cudaSuccess) return e;
+    decode_combine_kernel<__nv_bfloat16, 128><<<B * Hq, 128, 0, st>>>(part_o, part_ml, ns, (__nv_bfloat16 *)out,
+                                                                      lse);
+    return cudaGetLastError();
+  }
+  const DecodePlan pl = decode_plan(B, Hq, Hkv, D, max_seqlen, elem);
   CUtensorMap mK, mV;
   if (!make_cache_map(&mK, kc, B * Lcap, Hkv, D, elem) || !make_cache_map(&mV, vc, B * Lcap, Hkv, D, elem))
     return cudaErrorInvalidValue;

@@ -1,0 +1,549 @@
+// Tensor-core split-KV decode kernel for Dynamic Bifocal RoPE attention
+// (sm_100a, bf16, head_dim 128, up to 8 query heads per kv head).
+//
+// One generation step against a standard-RoPE cache that is never rewritten
+// (Jet-Long technical summary, §2 "Rotação de Correção On-the-Fly"): local
+// keys (L-1 - j < w0) keep the base RoPE, remote keys are scored at grouped
+// positions.  Rotations compose additively, so
+//     <R(delta_i) q~, R(delta_j) k~_j> = <q~, R(delta_j - delta_i) k~_j>:
+// each remote key row is rotated once, by the relative shift, and the stored
+// query is used unchanged.
+//
+// CTA (split, kv head, sequence), 320 threads, keys [split*chunk, ...) in
+// tiles of 128:
+//   warp 8     TMA producer: K and V tiles (128 keys x 128 d, SWIZZLE_128B) in
+//              two 3-stage rings.
+//   warps 4-7  rotation warpgroup: rotates the remote rows of each K tile in
+//              shared memory by R(delta_j - delta_i); thread t owns one 16-byte
+//              column chunk (8 pairs) of rows t/8 + 16m, so its angles advance
+//              by a fixed 16-key stride (fp32 cos/sin recurrence, fp64 seed).
+//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer:
+//              S^T = K Q^T   (M = 128 keys, N = 16: the GQA heads, zero-padded)
+//              O^T += V^T P  (M = 128 = head_dim, N = 16, V read MN-major)
+//   warps 0-3  softmax warpgroup: thread r owns key r of the tile (S^T lane r)
+//              and head-dim row r of O^T; block-wide running max per head,
+//              P written to shared memory as the B operand of the PV MMA, lazy
+//              O rescale, the CTA's partial (m, l, O) at the end.
+// The splits are merged by decode_combine_kernel (jl_decode.cu).  Every
+// mbarrier wait is bounded; on expiry the kernel records an error bit in the
+// workspace, stops the other roles, drains its own copies and MMAs, frees
+// TMEM and returns.
+#include "jl_common.cuh"
+#include "jl_ptx.cuh"
+
+namespace jl {
+namespace dtc {
+
+constexpr int THREADS = 320;
+constexpr int TK = 128;   // keys per tile
+constexpr int HD = 128;   // head_dim
+constexpr int NKS = 3;    // K ring stages
+constexpr int NVS = 3;    // V ring stages
+constexpr int TILE_BYTES = TK * HD * 2;
+constexpr int HALF_BYTES = TILE_BYTES / 2;
+constexpr int OPB = 16 * 128 * 2;  // a 16-row operand (Q or P): 2 halves x 16 rows x 128 B
+constexpr int OFF_K = 0;
+constexpr int OFF_V = NKS * TILE_BYTES;
+constexpr int OFF_Q = OFF_V + NVS * TILE_BYTES;
+constexpr int OFF_P = OFF_Q + OPB;
+constexpr int SMEM_USED = OFF_P + 2 * OPB;
+constexpr int SMEM_ALLOC = SMEM_USED + 1024;
+constexpr uint32_t TMEM_COLS = 64;  // S^T 0: [0,16), S^T 1: [16,32), O^T: [32,48)
+constexpr uint32_t COL_O = 32;
+constexpr int ERR_TIMEOUT = 16;
+// kind::f16, D fp32, A/B bf16, M = 128, N = 16; PV reads A (= V^T) MN-major
+constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 15);
+
+struct Args {
+  const __nv_bfloat16 *q;
+  const int32_t *seqlens;
+  int Lcap, Hq, Hkv;
+  long long w_pre;
+  int w0, plain, chunk, nsplit;
+  float *part_o, *part_ml;
+  int *err;
+};
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {  // K-major, SWIZZLE_128B
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr, uint32_t lbo) {  // MN-major, SWIZZLE_128B
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// byte offset of (row, 16-byte chunk) in a 16-row K-major SWIZZLE_128B operand
+// half (rows 128 B apart, chunk XOR-swizzled by row % 8)
+__device__ __forceinline__ int op_off(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+template <int GS>
+__global__ void __launch_bounds__(THREADS, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+                 const __grid_constant__ Args p, const __grid_constant__ InvFreq inv) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_kf[NKS], bar_kr[NKS], bar_ke[NKS], bar_vf[NVS], bar_ve[NVS], bar_sf[2],
+      bar_pr[2], bar_q, bar_od, bar_drain, bar_red[2], bar_lred;
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+  __shared__ float red[2][4][8];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  int L = p.seqlens[b];
+  if (L < 0 || L > p.Lcap || L > p.nsplit * p.chunk) L = 0;  // never read past the cache
+  const int kb = split * p.chunk;
+  const int ke = min(L, kb + p.chunk);
+  const int n = max(0, ke - kb);
+  const size_t pidx = ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;  // + g * nsplit
+  if (n == 0) {
+    for (int idx = threadIdx.x; idx < GS * HD; idx += THREADS)
+      p.part_o[(pidx + (size_t)(idx / HD) * p.nsplit) * HD + idx % HD] = 0.f;
+    if (threadIdx.x < GS) {
+      p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 0] = -INFINITY;
+      p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 1] = 0.f;
+    }
+    return;
+  }
+  const int ntiles = (n + TK - 1) / TK;
+  const int row0 = b * p.Lcap + kb;
+  const int i = L - 1;
+  const int G = p.plain ? 1 : (int)group_size(L, p.w_pre);
+  const bool bif = G > 1;
+  const int j_local = (int)max(0LL, (long long)L - (long long)p.w0);  // keys >= j_local are local
+
+  const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NKS; ++s) {
+      mbar_init(&bar_kf[s], 1);
+      mbar_init(&bar_kr[s], 128);
+      mbar_init(&bar_ke[s], 1);
+    }
+    for (int s = 0; s < NVS; ++s) {
+      mbar_init(&bar_vf[s], 1);
+      mbar_init(&bar_ve[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar_sf[s], 1);
+      mbar_init(&bar_pr[s], 128);
+    }
+    mbar_init(&bar_q, 128);
+    mbar_init(&bar_red[0], 4);
+    mbar_init(&bar_red[1], 4);
+    mbar_init(&bar_lred, 4);
+    mbar_init(&bar_od, 1);
+    mbar_init(&bar_drain, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 8) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      int nk = 0, nv = 0;
+      bool ok = true;
+      for (int u = 0; u < ntiles && ok; ++u) {
+        const int sk = u % NKS, sv = u % NVS;
+        if (u >= NKS && !(ok = wait_b(&bar_ke[sk], ((u / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT))) break;
+        mbar_expect_tx(&bar_kf[sk], TILE_BYTES);
+        tma_load(&mK, &bar_kf[sk], sbase + OFF_K + sk * TILE_BYTES, 0, kvh, row0 + u * TK);
+        tma_load(&mK, &bar_kf[sk], sbase + OFF_K + sk * TILE_BYTES + HALF_BYTES, 64, kvh, row0 + u * TK);
+        ++nk;
+        if (u >= NVS && !(ok = wait_b(&bar_ve[sv], ((u / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT))) break;
+        mbar_expect_tx(&bar_vf[sv], TILE_BYTES);
+        tma_load(&mV, &bar_vf[sv], sbase + OFF_V + sv * TILE_BYTES, 0, kvh, row0 + u * TK);
+        tma_load(&mV, &bar_vf[sv], sbase + OFF_V + sv * TILE_BYTES + HALF_BYTES, 64, kvh, row0 + u * TK);
+        ++nv;
+      }
+      for (int u = max(0, nk - NKS); u < nk; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT);
+      for (int u = max(0, nv - NVS); u < nv; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT);
+    }
+  } else if (warp == 9) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT);
+      int u = 0;
+      auto issue_pv = [&](int w) -> bool {
+        const int sv = w % NVS;
+        if (!wait_b(&bar_vf[sv], (w / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT)) return false;
+        if (!wait_b(&bar_pr[w & 1], (w >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT)) return false;
+        fence_after();
+        const uint32_t va = sbase + OFF_V + sv * TILE_BYTES;
+        const uint32_t pa = sbase + OFF_P + (w & 1) * OPB;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + COL_O, desc_mn(va + kk * 2048, HALF_BYTES),
+                 desc_k(pa + (kk >> 2) * (OPB / 2) + (kk & 3) * 32), IDESC_PV, (w > 0 || kk > 0) ? 1u : 0u);
+        commit(&bar_ve[sv]);
+        commit(&bar_od);
+        return true;
+      };
+      for (; u < ntiles && ok; ++u) {
+        const int sk = u % NKS;
+        if (!(ok = wait_b(&bar_kr[sk], (u / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT))) break;
+        fence_after();
+        const uint32_t ka = sbase + OFF_K + sk * TILE_BYTES;
+        const uint32_t qa = sbase + OFF_Q;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t ko = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          const uint32_t qo = (kk >> 2) * (OPB / 2) + (kk & 3) * 32;
+          mma_ss(tmem + (uint32_t)((u & 1) * 16), desc_k(ka + ko), desc_k(qa + qo), IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        commit(&bar_sf[u & 1]);
+        commit(&bar_ke[sk]);
+        if (u > 0 && !(ok = issue_pv(u - 1))) break;
+      }
+      if (ok && u > 0) issue_pv(u - 1);
+      commit(&bar_drain);
+      wait_drain(&bar_drain, 0, p.err, ERR_TIMEOUT);
+    }
+  } else if (warp >= 4) {
+    // ======================= rotation warpgroup =======================
+    const int t = threadIdx.x - 128;
+    const int pc = t & 7;           // physical 16-byte chunk within a 128-byte row
+    const int r0 = t >> 3;          // first row (0..15); rows r0 + 16m
+    const int lc = pc ^ (r0 & 7);   // logical chunk: pairs k = 8 lc .. 8 lc + 7
+    float ec[8], es[8], w1c[8], w1s[8], w0c[8], w0s[8];
+    int rm = 0;
+    const int stride_full = 16 - 16 / G;  // n(j + 16) - n(j) without a carry
+    const int smod = 16 % G;
+    if (bif) {
+      const int jf = kb + r0;
+      const int ni = corr_n(i, G);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const double w = inv.v[lc * 8 + e];
+        angle_cs(corr_n(jf, G) - ni, w, ec[e], es[e]);
+        angle_cs(stride_full, w, w1c[e], w1s[e]);
+        angle_cs(stride_full - 1, w, w0c[e], w0s[e]);
+      }
+      rm = jf % G;
+    }
+    bool ok = true;
+    for (int u = 0; u < ntiles && ok; ++u) {
+      const int sk = u % NKS;
+      ok = __all_sync(0xffffffffu, wait_b(&bar_kf[sk], (u / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+      if (!ok) break;
+      const int j0 = kb + u * TK;
+      if (bif && j0 < j_local) {
+        uint8_t *kt = gbase + OFF_K + sk * TILE_BYTES;
+#pragma unroll 2
+        for (int m = 0; m < 8; ++m) {
+          const int r = r0 + 16 * m;
+          if (j0 + r < j_local) {
+            uint4 *pa = reinterpret_cast<uint4 *>(kt + r * 128 + pc * 16);
+            uint4 *pb = reinterpret_cast<uint4 *>(kt + HALF_BYTES + r * 128 + pc * 16);
+            uint4 xa = *pa, xb = *pb;
+            uint32_t *ua = reinterpret_cast<uint32_t *>(&xa), *ub = reinterpret_cast<uint32_t *>(&xb);
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&ua[e2]));
+              float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&ub[e2]));
+              rot_back(fa.x, fb.x, ec[2 * e2], es[2 * e2]);
+              rot_back(fa.y, fb.y, ec[2 * e2 + 1], es[2 * e2 + 1]);
+              __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
+              __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
+              ua[e2] = *reinterpret_cast<uint32_t *>(&ra);
+              ub[e2] = *reinterpret_cast<uint32_t *>(&rb);
+            }
+            *pa = xa;
+            *pb = xb;
+          }
+          // advance to key j + 16: n grows by 16 - floor((j+16)/G) + floor(j/G)
+          rm += smod;
+          const bool carry = rm >= G;
+          if (carry) rm -= G;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float wc = carry ? w0c[e] : w1c[e];
+            const float ws = carry ? w0s[e] : w1s[e];
+            const float c2 = ec[e] * wc - es[e] * ws;
+            const float s2 = es[e] * wc + ec[e] * ws;
+            ec[e] = c2;
+            es[e] = s2;
+          }
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      } else if (bif) {
+        // no remote key in this tile: only advance the recurrence by 8 rows
+#pragma unroll 1
+        for (int m = 0; m < 8; ++m) {
+          rm += smod;
+          const bool carry = rm >= G;
+          if (carry) rm -= G;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float wc = carry ? w0c[e] : w1c[e];
+            const float ws = carry ? w0s[e] : w1s[e];
+            const float c2 = ec[e] * wc - es[e] * ws;
+            const float s2 = es[e] * wc + ec[e] * ws;
+            ec[e] = c2;
+            es[e] = s2;
+          }
+        }
+      }
+      mbar_arrive(&bar_kr[sk]);
+    }
+  } else {
+    // ======================= softmax warpgroup =======================
+    const int r = threadIdx.x;  // key row of the tile / head-dim row of O^T / TMEM lane
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;
+    // Q operand: rows h < GS hold the query heads, rows GS..15 zero; also zero
+    // the padding rows of both P buffers
+    {
+      const int h = r >> 3, c = r & 7;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (h < GS)
+          val = *reinterpret_cast<const uint4 *>(p.q + ((size_t)b * p.Hq + (size_t)kvh * GS + h) * HD + hf * 64 +
+                                                 c * 8);
+        *reinterpret_cast<uint4 *>(gbase + OFF_Q + hf * (OPB / 2) + op_off(h, c)) = val;
+        if (h >= GS)
+#pragma unroll
+          for (int pb = 0; pb < 2; ++pb)
+            *reinterpret_cast<uint4 *>(gbase + OFF_P + pb * OPB + hf * (OPB / 2) + op_off(h, c)) =
+                make_uint4(0u, 0u, 0u, 0u);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bar_q);
+    }
+    float m_run[GS], l_part[GS];
+#pragma unroll
+    for (int g = 0; g < GS; ++g) {
+      m_run[g] = -INFINITY;
+      l_part[g] = 0.f;
+    }
+    bool ok = true;
+    int u = 0;
+    for (; u < ntiles && ok; ++u) {
+      const int bsel = u & 1;
+      ok = __all_sync(0xffffffffu, wait_b(&bar_sf[bsel], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+      if (!ok) break;
+      fence_after();
+      uint32_t sr[8];
+      tmem_ld8(tmem + lane_base + (uint32_t)(bsel * 16), sr);
+      const int j = kb + u * TK + r;
+      const bool valid = j < ke;
+      float s[GS];
+#pragma unroll
+      for (int g = 0; g < GS; ++g) s[g] = valid ? __uint_as_float(sr[g]) * sl2 : -INFINITY;
+      // block-wide tile max per head
+      float mt[GS];
+#pragma unroll
+      for (int g = 0; g < GS; ++g) {
+        float x = s[g];
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+        mt[g] = x;
+      }
+      // exchange the four warps' maxima through shared memory (an mbarrier
+      // with one arrival per warp, waited with a bound)
+      if (lane == 0) {
+#pragma unroll
+        for (int g = 0; g < GS; ++g) red[bsel][warp][g] = mt[g];
+        mbar_arrive(&bar_red[bsel]);
+      }
+      ok = __all_sync(0xffffffffu, wait_b(&bar_red[bsel], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+      if (!ok) break;
+#pragma unroll
+      for (int g = 0; g < GS; ++g)
+        mt[g] = fmaxf(fmaxf(red[bsel][0][g], red[bsel][1][g]), fmaxf(red[bsel][2][g], red[bsel][3][g]));
+      // lazy rescale: only when a head's max grows by more than 2^8
+      float f[GS];
+      bool any = false;
+#pragma unroll
+      for (int g = 0; g < GS; ++g) {
+        const float mn = fmaxf(m_run[g], mt[g]);
+        f[g] = 1.f;
+        if (m_run[g] == -INFINITY) {
+          m_run[g] = mn;
+        } else if (mn > m_run[g] + 8.f) {
+          f[g] = exp2f(m_run[g] - mn);
+          m_run[g] = mn;
+          any = true;
+        }
+      }
+      if (any) {  // uniform over the warpgroup (all threads see the same maxima)
+        ok = __all_sync(0xffffffffu, wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+        if (!ok) break;
+        fence_after();
+        uint32_t orow[8];
+        tmem_ld8(tmem + lane_base + COL_O, orow);
+#pragma unroll
+        for (int g = 0; g < GS; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * f[g]);
+        tmem_st8(tmem + lane_base + COL_O, orow);
+#pragma unroll
+        for (int g = 0; g < GS; ++g) l_part[g] *= f[g];
+      }
+      // P (bf16) into the B operand of the PV MMA: row g = head, column r = key
+      uint8_t *pbuf = gbase + OFF_P + bsel * OPB + (r >> 6) * (OPB / 2);
+      const int chunk = (r & 63) >> 3;
+#pragma unroll
+      for (int g = 0; g < GS; ++g) {
+        const float pr = valid ? ex2(s[g] - m_run[g]) : 0.f;
+        l_part[g] += pr;
+        *reinterpret_cast<__nv_bfloat16 *>(pbuf + op_off(g, chunk) + (r & 7) * 2) = __float2bfloat16_rn(pr);
+      }
+      // a partial last tile: zero the V rows past the last key (the cache may
+      // hold anything there, and 0 * NaN would poison the PV product)
+      if (u == ntiles - 1 && (n % TK) != 0) {
+        const int sv = u % NVS;
+        ok = __all_sync(0xffffffffu, wait_b(&bar_vf[sv], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+        if (!ok) break;
+        if (!valid) {
+          uint8_t *vt = gbase + OFF_V + sv * TILE_BYTES;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            *reinterpret_cast<uint4 *>(vt + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(vt + HALF_BYTES + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      }
+      // last tile: PV of the previous tile must be complete before this
+      // tile's PV is released, so exactly one PV is outstanding at the end
+      if (u == ntiles - 1 && u > 0) {
+        ok = __all_sync(0xffffffffu, wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+        if (!ok) break;
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      fence_before();
+      mbar_arrive(&bar_pr[bsel]);
+    }
+    // ---- epilogue: this split's partial (m, l, O) per head
+    if (ok && u > 0) ok = __all_sync(0xffffffffu, wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+    float lsum[GS];
+#pragma unroll
+    for (int g = 0; g < GS; ++g) {
+      float x = l_part[g];
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      lsum[g] = x;
+    }
+    __shared__ float lred[4][8];
+    if (lane == 0) {
+#pragma unroll
+      for (int g = 0; g < GS; ++g) lred[warp][g] = lsum[g];
+      mbar_arrive(&bar_lred);
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_b(&bar_lred, 0, &abort_flag, p.err, ERR_TIMEOUT));
+    if (ok) {
+      fence_after();
+      uint32_t orow[8];
+      tmem_ld8(tmem + lane_base + COL_O, orow);
+#pragma unroll
+      for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * HD + r] = __uint_as_float(orow[g]);
+      if (r < GS) {
+        const float l = lred[0][r] + lred[1][r] + lred[2][r] + lred[3][r];
+        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 0] = m_run[r];
+        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 1] = l;
+      }
+    } else {
+      for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * HD + r] = 0.f;
+      if (r < GS) {
+        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 0] = -INFINITY;
+        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 1] = 0.f;
+      }
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
+}  // namespace dtc
+
+// ------------------------------------------------------------------ host
+// Split plan: one CTA per SM (the rings take ~200 KB of shared memory), one
+// wave of 148, whole 128-key tiles.
+void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk) {
+  const int ns0 = max(1, 148 / max(1, batch * Hkv));
+  const int maxL = max(1, max_seqlen);
+  int c = (maxL + ns0 - 1) / ns0;
+  c = (c + dtc::TK - 1) / dtc::TK * dtc::TK;
+  *chunk = c;
+  *nsplit = (maxL + c - 1) / c;
+}
+
+cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
+                             const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
+                             const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o, float *part_ml,
+                             int *err, cudaStream_t st) {
+  dtc::Args a;
+  a.q = q;
+  a.seqlens = seqlens;
+  a.Lcap = Lcap;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.w_pre = w_pre;
+  a.w0 = w0;
+  a.plain = plain;
+  a.chunk = chunk;
+  a.nsplit = nsplit;
+  a.part_o = part_o;
+  a.part_ml = part_ml;
+  a.err = err;
+  dim3 grid(nsplit, Hkv, B);
+  cudaError_t e;
+#define JL_DTC(GG)                                                                                       \
+  e = cudaFuncSetAttribute(dtc::decode_tc_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,         \
+                           dtc::SMEM_ALLOC);                                                              \
+  if (e != cudaSuccess) return e;                                                                        \
+  dtc::decode_tc_kernel<GG><<<grid, dtc::THREADS, dtc::SMEM_ALLOC, st>>>(mK, mV, a, inv);
+  switch (GS) {
+    case 1: JL_DTC(1) break;
+    case 2: JL_DTC(2) break;
+    case 4: JL_DTC(4) break;
+    case 8: JL_DTC(8) break;
+    default: return cudaErrorInvalidValue;
+  }
+#undef JL_DTC
+  return cudaGetLastError();
+}
+
+}  // namespace jl

@@ -74,6 +74,12 @@ __device__ __forceinline__ void tma_load(const CUtensorMap *map, uint64_t *bar, 
       : "memory");
 }
 
+__device__ __forceinline__ float ex2(float x) {  // MUFU exp2 (ex2.approx.ftz)
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Host: cuTensorMapEncodeTiled through the runtime's driver entry point (no
 // link-time dependency on libcuda).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
