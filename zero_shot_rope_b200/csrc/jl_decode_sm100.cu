@@ -9,17 +9,17 @@
 // each remote key row is rotated once, by the relative shift, and the stored
 // query is used unchanged.
 //
-// CTA (split, kv head, sequence), 320 threads, keys [split*chunk, ...) in
+// CTA (split, kv head, sequence), 448 threads, keys [split*chunk, ...) in
 // tiles of 128:
-//   warp 8     TMA producer: K and V tiles (128 keys x 128 d, SWIZZLE_128B) in
+//   warp 12    TMA producer: K and V tiles (128 keys x 128 d, SWIZZLE_128B) in
 //              two 3-stage rings.
-//   warps 4-7  rotation warpgroup: rotates the remote rows of each K tile in
-//              shared memory by R(delta_j - delta_i); thread t owns one 16-byte
-//              column chunk (8 pairs) of rows t/8 + 16m, so its angles advance
-//              by a fixed 16-key stride (fp32 cos/sin recurrence, fp64 seed).
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer:
+//   warps 4-11 rotation warps: rotate the remote rows of each K tile in shared
+//              memory by R(delta_j - delta_i); thread t owns one 16-byte column
+//              chunk (8 pairs) of rows t/8 + 32m, so its angles advance by a
+//              fixed 32-key stride (fp32 cos/sin recurrence, fp64 seed).
+//   warp 13    TMEM allocator and single-thread tcgen05.mma issuer, per tile
 //              S^T = K Q^T   (M = 128 keys, N = 16: the GQA heads, zero-padded)
-//              O^T += V^T P  (M = 128 = head_dim, N = 16, V read MN-major)
+//              then O^T += V^T P  (M = 128 = head_dim, N = 16, V read MN-major)
 //   warps 0-3  softmax warpgroup: thread r owns key r of the tile (S^T lane r)
 //              and head-dim row r of O^T; block-wide running max per head,
 //              P written to shared memory as the B operand of the PV MMA, lazy
@@ -34,9 +34,14 @@
 namespace jl {
 namespace dtc {
 
-constexpr int THREADS = 320;
 constexpr int TK = 128;   // keys per tile
 constexpr int HD = 128;   // head_dim
+constexpr int NROT = 8;                          // rotation warps
+constexpr int THREADS = 128 + NROT * 32 + 64;   // softmax + rotation + TMA + MMA
+constexpr int WARP_TMA = 4 + NROT;
+constexpr int WARP_MMA = 5 + NROT;
+constexpr int ROT_ROWS = TK * 8 / (NROT * 32);  // rows per rotation thread per tile
+
 constexpr int NKS = 3;    // K ring stages
 constexpr int NVS = 3;    // V ring stages
 constexpr int TILE_BYTES = TK * HD * 2;
@@ -111,7 +116,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
                  const __grid_constant__ Args p, const __grid_constant__ InvFreq inv) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_kf[NKS], bar_kr[NKS], bar_ke[NKS], bar_vf[NVS], bar_ve[NVS], bar_sf[2],
-      bar_pr[2], bar_q, bar_od, bar_drain, bar_red[2], bar_lred;
+      bar_pr[2], bar_q, bar_od, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   __shared__ float red[2][4][8];
@@ -146,7 +151,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   if (threadIdx.x == 0) {
     for (int s = 0; s < NKS; ++s) {
       mbar_init(&bar_kf[s], 1);
-      mbar_init(&bar_kr[s], 128);
+      mbar_init(&bar_kr[s], NROT * 32);
       mbar_init(&bar_ke[s], 1);
     }
     for (int s = 0; s < NVS; ++s) {
@@ -158,15 +163,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       mbar_init(&bar_pr[s], 128);
     }
     mbar_init(&bar_q, 128);
-    mbar_init(&bar_red[0], 4);
-    mbar_init(&bar_red[1], 4);
-    mbar_init(&bar_lred, 4);
     mbar_init(&bar_od, 1);
     mbar_init(&bar_drain, 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 9) {
+  if (warp == WARP_MMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_slot)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -176,7 +178,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   fence_after();
   const uint32_t tmem = tmem_slot;
 
-  if (warp == 8) {
+  if (warp == WARP_TMA) {
     // ======================= TMA producer =======================
     if (lane == 0) {
       int nk = 0, nv = 0;
@@ -197,56 +199,75 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       for (int u = max(0, nk - NKS); u < nk; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT);
       for (int u = max(0, nv - NVS); u < nv; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT);
     }
-  } else if (warp == 9) {
+  } else if (warp == WARP_MMA) {
     // ======================= MMA issuer =======================
+    // A small scheduler: QK of tile uq as soon as its rotated K is ready (and
+    // its S buffer is free, i.e. PV of tile uq-2 issued), PV of tile up as
+    // soon as its P and V are ready.  Neither waits on the other's inputs.
     if (lane == 0) {
       bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT);
-      int u = 0;
-      auto issue_pv = [&](int w) -> bool {
-        const int sv = w % NVS;
-        if (!wait_b(&bar_vf[sv], (w / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT)) return false;
-        if (!wait_b(&bar_pr[w & 1], (w >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT)) return false;
-        fence_after();
-        const uint32_t va = sbase + OFF_V + sv * TILE_BYTES;
-        const uint32_t pa = sbase + OFF_P + (w & 1) * OPB;
+      int uq = 0, up = 0;
+      uint64_t t_idle = gtime();
+      uint32_t spins = 0;
+      while (ok && up < ntiles) {
+        bool progressed = false;
+        if (uq < ntiles && uq - up < 2 && mbar_test(&bar_kr[uq % NKS], (uq / NKS) & 1)) {
+          fence_after();
+          const int sk = uq % NKS;
+          const uint32_t ka = sbase + OFF_K + sk * TILE_BYTES;
+          const uint32_t qa = sbase + OFF_Q;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + COL_O, desc_mn(va + kk * 2048, HALF_BYTES),
-                 desc_k(pa + (kk >> 2) * (OPB / 2) + (kk & 3) * 32), IDESC_PV, (w > 0 || kk > 0) ? 1u : 0u);
-        commit(&bar_ve[sv]);
-        commit(&bar_od);
-        return true;
-      };
-      for (; u < ntiles && ok; ++u) {
-        const int sk = u % NKS;
-        if (!(ok = wait_b(&bar_kr[sk], (u / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT))) break;
-        fence_after();
-        const uint32_t ka = sbase + OFF_K + sk * TILE_BYTES;
-        const uint32_t qa = sbase + OFF_Q;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t ko = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * (OPB / 2) + (kk & 3) * 32;
-          mma_ss(tmem + (uint32_t)((u & 1) * 16), desc_k(ka + ko), desc_k(qa + qo), IDESC_QK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t ko = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+            const uint32_t qo = (kk >> 2) * (OPB / 2) + (kk & 3) * 32;
+            mma_ss(tmem + (uint32_t)((uq & 1) * 16), desc_k(ka + ko), desc_k(qa + qo), IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          commit(&bar_sf[uq & 1]);
+          commit(&bar_ke[sk]);
+          ++uq;
+          progressed = true;
         }
-        commit(&bar_sf[u & 1]);
-        commit(&bar_ke[sk]);
-        if (u > 0 && !(ok = issue_pv(u - 1))) break;
+        if (up < uq && mbar_test(&bar_pr[up & 1], (up >> 1) & 1) &&
+            mbar_test(&bar_vf[up % NVS], (up / NVS) & 1)) {
+          fence_after();
+          const int sv = up % NVS;
+          const uint32_t va = sbase + OFF_V + sv * TILE_BYTES;
+          const uint32_t pa = sbase + OFF_P + (up & 1) * OPB;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tmem + COL_O, desc_mn(va + kk * 2048, HALF_BYTES),
+                   desc_k(pa + (kk >> 2) * (OPB / 2) + (kk & 3) * 32), IDESC_PV, (up > 0 || kk > 0) ? 1u : 0u);
+          commit(&bar_ve[sv]);
+          commit(&bar_od);
+          ++up;
+          progressed = true;
+        }
+        if (progressed) {
+          spins = 0;
+          t_idle = gtime();
+        } else if ((++spins & 31u) == 0) {
+          if (abort_flag) ok = false;
+          else if (gtime() - t_idle > 2000000000ull) {
+            abort_flag = 1;
+            atomicOr(p.err, ERR_TIMEOUT);
+            ok = false;
+          }
+        }
       }
-      if (ok && u > 0) issue_pv(u - 1);
       commit(&bar_drain);
       wait_drain(&bar_drain, 0, p.err, ERR_TIMEOUT);
     }
   } else if (warp >= 4) {
-    // ======================= rotation warpgroup =======================
+    // ======================= rotation warps =======================
+    constexpr int RS = TK / ROT_ROWS;  // row stride of one thread (32)
     const int t = threadIdx.x - 128;
     const int pc = t & 7;           // physical 16-byte chunk within a 128-byte row
-    const int r0 = t >> 3;          // first row (0..15); rows r0 + 16m
+    const int r0 = t >> 3;          // first row (0..RS-1); rows r0 + RS m
     const int lc = pc ^ (r0 & 7);   // logical chunk: pairs k = 8 lc .. 8 lc + 7
     float ec[8], es[8], w1c[8], w1s[8], w0c[8], w0s[8];
     int rm = 0;
-    const int stride_full = 16 - 16 / G;  // n(j + 16) - n(j) without a carry
-    const int smod = 16 % G;
+    const int stride_full = RS - RS / G;  // n(j + RS) - n(j) without a carry
+    const int smod = RS % G;
     if (bif) {
       const int jf = kb + r0;
       const int ni = corr_n(i, G);
@@ -267,9 +288,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       const int j0 = kb + u * TK;
       if (bif && j0 < j_local) {
         uint8_t *kt = gbase + OFF_K + sk * TILE_BYTES;
-#pragma unroll 2
-        for (int m = 0; m < 8; ++m) {
-          const int r = r0 + 16 * m;
+#pragma unroll
+        for (int m = 0; m < ROT_ROWS; ++m) {
+          const int r = r0 + RS * m;
           if (j0 + r < j_local) {
             uint4 *pa = reinterpret_cast<uint4 *>(kt + r * 128 + pc * 16);
             uint4 *pb = reinterpret_cast<uint4 *>(kt + HALF_BYTES + r * 128 + pc * 16);
@@ -289,7 +310,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
             *pa = xa;
             *pb = xb;
           }
-          // advance to key j + 16: n grows by 16 - floor((j+16)/G) + floor(j/G)
+          // advance to key j + RS: n grows by RS - floor((j+RS)/G) + floor(j/G)
           rm += smod;
           const bool carry = rm >= G;
           if (carry) rm -= G;
@@ -305,9 +326,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       } else if (bif) {
-        // no remote key in this tile: only advance the recurrence by 8 rows
+        // no remote key in this tile: only advance the recurrence
 #pragma unroll 1
-        for (int m = 0; m < 8; ++m) {
+        for (int m = 0; m < ROT_ROWS; ++m) {
           rm += smod;
           const bool carry = rm >= G;
           if (carry) rm -= G;
@@ -359,8 +380,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     int u = 0;
     for (; u < ntiles && ok; ++u) {
       const int bsel = u & 1;
-      ok = __all_sync(0xffffffffu, wait_b(&bar_sf[bsel], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
-      if (!ok) break;
+      // on a timeout this warp carries on with garbage until the barrier below,
+      // where every warp of the group sees the abort and leaves together
+      wait_b(&bar_sf[bsel], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT);
       fence_after();
       uint32_t sr[8];
       tmem_ld8(tmem + lane_base + (uint32_t)(bsel * 16), sr);
@@ -378,15 +400,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
         mt[g] = x;
       }
-      // exchange the four warps' maxima through shared memory (an mbarrier
-      // with one arrival per warp, waited with a bound)
-      if (lane == 0) {
+      // exchange the four warps' maxima through shared memory; the named
+      // barrier also ORs the abort state so that all four warps leave the
+      // loop at the same tile (keeping their barrier counts equal)
+      if (lane == 0)
 #pragma unroll
         for (int g = 0; g < GS; ++g) red[bsel][warp][g] = mt[g];
-        mbar_arrive(&bar_red[bsel]);
+      if (bar_red_or(1, 128, abort_flag != 0)) {
+        ok = false;
+        break;
       }
-      ok = __all_sync(0xffffffffu, wait_b(&bar_red[bsel], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
-      if (!ok) break;
 #pragma unroll
       for (int g = 0; g < GS; ++g)
         mt[g] = fmaxf(fmaxf(red[bsel][0][g], red[bsel][1][g]), fmaxf(red[bsel][2][g], red[bsel][3][g]));
@@ -406,8 +429,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         }
       }
       if (any) {  // uniform over the warpgroup (all threads see the same maxima)
-        ok = __all_sync(0xffffffffu, wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
-        if (!ok) break;
+        // O holds PV of tiles < u once PV_{u-1} is complete
+        wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT);
         fence_after();
         uint32_t orow[8];
         tmem_ld8(tmem + lane_base + COL_O, orow);
@@ -430,9 +453,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       // hold anything there, and 0 * NaN would poison the PV product)
       if (u == ntiles - 1 && (n % TK) != 0) {
         const int sv = u % NVS;
-        ok = __all_sync(0xffffffffu, wait_b(&bar_vf[sv], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT));
-        if (!ok) break;
-        if (!valid) {
+        wait_b(&bar_vf[sv], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT);
+        if (!valid && !abort_flag) {
           uint8_t *vt = gbase + OFF_V + sv * TILE_BYTES;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -443,16 +465,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       }
       // last tile: PV of the previous tile must be complete before this
       // tile's PV is released, so exactly one PV is outstanding at the end
-      if (u == ntiles - 1 && u > 0) {
-        ok = __all_sync(0xffffffffu, wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
-        if (!ok) break;
-      }
+      if (u == ntiles - 1 && u > 0) wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       fence_before();
       mbar_arrive(&bar_pr[bsel]);
     }
     // ---- epilogue: this split's partial (m, l, O) per head
-    if (ok && u > 0) ok = __all_sync(0xffffffffu, wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT));
+    if (ok && u > 0) wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT);
     float lsum[GS];
 #pragma unroll
     for (int g = 0; g < GS; ++g) {
@@ -462,12 +481,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       lsum[g] = x;
     }
     __shared__ float lred[4][8];
-    if (lane == 0) {
+    if (lane == 0)
 #pragma unroll
       for (int g = 0; g < GS; ++g) lred[warp][g] = lsum[g];
-      mbar_arrive(&bar_lred);
-    }
-    if (ok) ok = __all_sync(0xffffffffu, wait_b(&bar_lred, 0, &abort_flag, p.err, ERR_TIMEOUT));
+    if (bar_red_or(1, 128, abort_flag != 0)) ok = false;
     if (ok) {
       fence_after();
       uint32_t orow[8];
@@ -490,7 +507,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
 
   fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == WARP_MMA) {
     fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
   }
