@@ -31,6 +31,8 @@
 // its own copies and MMAs in flight, frees TMEM and returns.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "jl_common.cuh"
 #include "jl_ptx.cuh"
 
@@ -120,6 +122,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       JL_W32(r)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 // wait::ld that also "redefines" the loaded registers, so no use of them can be
 // scheduled before the wait
@@ -156,27 +166,58 @@ struct Tile {
   int L, G, i0, i1, qt, bif;
 };
 
-// Visits of key tile kt: up to two (grouped part, base part).  For each,
-// columns c with (i - j0 - c) in [lo, hi] are kept when `mask` is set.
+// Visits of a query tile, in order: the grouped visits (key tiles whose
+// pairs include a distance >= w0) on key tiles 0 .. kg_end-1, then the base
+// visits (pairs with distance < w0) on key tiles ks_begin .. qt.  A visit's
+// columns c with (i - j0 - c) outside [lo, hi] are masked when `mask` is set.
+// The diagonal tile is always masked: besides j > i it holds the keys at or
+// past L (zero-filled, or the next sequence's).  Everything is computed from
+// integers in registers (no per-visit arrays).
 struct Visit {
   int grp, mask, lo, hi;
 };
 
-__device__ __forceinline__ int visits_of(const Tile &t, int w0, int kt, Visit (&vs)[2]) {
+struct VisitPlan {
+  int n_grp, n_all, ks_begin;
+};
+
+__device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
+  VisitPlan pl;
+  if (!t.bif) {
+    pl.n_grp = 0;
+    pl.ks_begin = 0;
+    pl.n_all = t.qt + 1;
+    return pl;
+  }
+  // grouped: dmax(kt) = i1 - kt*BN >= w0
+  pl.n_grp = (t.i1 >= w0) ? min(t.qt, (t.i1 - w0) / BN) + 1 : 0;
+  // base: dmin(kt) <= w0 - 1; for kt < qt, dmin = i0 - kt*BN - (BN-1); the
+  // diagonal tile always qualifies when w0 >= 1
+  int nstd = 0;
+  pl.ks_begin = t.qt + 1;
+  if (w0 > 0) {
+    const int x = t.i0 - (BN - 1) - (w0 - 1);  // need kt*BN >= x
+    pl.ks_begin = x <= 0 ? 0 : min(t.qt, (x + BN - 1) / BN);
+    nstd = t.qt - pl.ks_begin + 1;
+  }
+  pl.n_all = pl.n_grp + nstd;
+  return pl;
+}
+
+__device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int w0, int v, int &kt, Visit &out) {
+  const bool grp = v < pl.n_grp;
+  kt = grp ? v : pl.ks_begin + (v - pl.n_grp);
   const int j0 = kt * BN;
   const int j1 = min(j0 + BN - 1, t.L - 1);
   const int dmin = t.i0 - j1, dmax = t.i1 - j0;
-  // the diagonal tile always needs the causal mask: besides j > i it holds
-  // the keys at or past L (zero-filled or the next sequence's)
   const int diag = kt == t.qt;
-  int n = 0;
-  if (!t.bif) {
-    vs[n++] = Visit{0, diag, 0, HI_INF};
-    return n;
+  if (grp) {
+    out = Visit{1, diag || dmin < w0, w0, HI_INF};
+  } else if (!t.bif) {
+    out = Visit{0, diag, 0, HI_INF};
+  } else {
+    out = Visit{0, diag || dmax > w0 - 1, 0, w0 - 1};
   }
-  if (dmax >= w0) vs[n++] = Visit{1, diag || dmin < w0, w0, HI_INF};
-  if (w0 > 0 && dmin <= w0 - 1) vs[n++] = Visit{0, diag || dmax > w0 - 1, 0, w0 - 1};
-  return n;
 }
 
 // ----------------------------------------------------------------- kernel
@@ -208,6 +249,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   t.bif = t.G > 1;
   const int kvh = h / (p.Hq / p.Hkv);
   const bool need_qg = t.bif && t.i1 >= p.w0;
+  const VisitPlan pl = make_plan(t, p.w0);
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
@@ -248,19 +290,18 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       tma_load(&mQ, &bar_q, sbase + OFF_Q + HALF_BYTES, 64, h, tok_q0);
       int v = 0;
       bool ok = true;
-      for (int kt = 0; kt <= t.qt && ok; ++kt) {
-        Visit vs[2];
-        const int nv = visits_of(t, p.w0, kt, vs);
-        for (int x = 0; x < nv; ++x, ++v) {
-          const int st = v % NKS;
-          if (v >= NKS && !(ok = wait_b(&bar_ke[st], ((v / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
-            break;
-          const CUtensorMap *m = vs[x].grp ? &mKg : &mK;
-          const uint32_t dst = sbase + OFF_K + st * TILE_BYTES;
-          mbar_expect_tx(&bar_kf[st], TILE_BYTES);
-          tma_load(m, &bar_kf[st], dst, 0, kvh, a + kt * BN);
-          tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
-        }
+      for (; v < pl.n_all; ++v) {
+        int kt;
+        Visit vx;
+        visit_at(t, pl, p.w0, v, kt, vx);
+        const int st = v % NKS;
+        if (v >= NKS && !(ok = wait_b(&bar_ke[st], ((v / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+          break;
+        const CUtensorMap *m = vx.grp ? &mKg : &mK;
+        const uint32_t dst = sbase + OFF_K + st * TILE_BYTES;
+        mbar_expect_tx(&bar_kf[st], TILE_BYTES);
+        tma_load(m, &bar_kf[st], dst, 0, kvh, a + kt * BN);
+        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
       }
       // drain: every load issued must land before the CTA may exit
       for (int u = max(0, v - NKS); u < v; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
@@ -271,18 +312,17 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     if (lane == 0) {
       int v = 0;
       bool ok = true;
-      for (int kt = 0; kt <= t.qt && ok; ++kt) {
-        Visit vs[2];
-        const int nv = visits_of(t, p.w0, kt, vs);
-        for (int x = 0; x < nv; ++x, ++v) {
-          const int st = v % NVS;
-          if (v >= NVS && !(ok = wait_b(&bar_ve[st], ((v / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
-            break;
-          const uint32_t dst = sbase + OFF_V + st * TILE_BYTES;
-          mbar_expect_tx(&bar_vf[st], TILE_BYTES);
-          tma_load(&mV, &bar_vf[st], dst, 0, kvh, a + kt * BN);
-          tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
-        }
+      for (; v < pl.n_all; ++v) {
+        int kt;
+        Visit vx;
+        visit_at(t, pl, p.w0, v, kt, vx);
+        const int st = v % NVS;
+        if (v >= NVS && !(ok = wait_b(&bar_ve[st], ((v / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+          break;
+        const uint32_t dst = sbase + OFF_V + st * TILE_BYTES;
+        mbar_expect_tx(&bar_vf[st], TILE_BYTES);
+        tma_load(&mV, &bar_vf[st], dst, 0, kvh, a + kt * BN);
+        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
       }
       for (int u = max(0, v - NVS); u < v; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
     }
@@ -307,18 +347,19 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         umma_commit(&bar_od);
         return true;
       };
-      for (int kt = 0; kt <= t.qt && ok; ++kt) {
-        Visit vs[2];
-        const int nv = visits_of(t, p.w0, kt, vs);
-        for (int x = 0; x < nv && ok; ++x, ++v) {
-          if (vs[x].grp && !qg_seen) {
+      for (; v < pl.n_all && ok; ++v) {
+        int kt;
+        Visit vx;
+        visit_at(t, pl, p.w0, v, kt, vx);
+        {
+          if (vx.grp && !qg_seen) {
             if (!(ok = wait_b(&bar_qg, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
             qg_seen = true;
           }
           const int st = v % NKS;
           if (!(ok = wait_b(&bar_kf[st], (v / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
           tc_fence_after();
-          const uint32_t qaddr = sbase + (vs[x].grp ? OFF_QG : OFF_Q);
+          const uint32_t qaddr = sbase + (vx.grp ? OFF_QG : OFF_Q);
           const uint32_t kaddr = sbase + OFF_K + st * TILE_BYTES;
           const uint32_t scol = tmem + (uint32_t)((v & 1) * 128);
 #pragma unroll
@@ -378,11 +419,12 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 
     float m_run = -INFINITY, l_run = 0.f;
     int v = 0;
-    for (int kt = 0; kt <= t.qt && ok; ++kt) {
-      Visit vs[2];
-      const int nv = visits_of(t, p.w0, kt, vs);
+    for (; v < pl.n_all && ok; ++v) {
+      int kt;
+      Visit vx;
+      visit_at(t, pl, p.w0, v, kt, vx);
       const int dc = i - kt * BN;  // column c has distance dc - c
-      for (int x = 0; x < nv && ok; ++x, ++v) {
+      {
         const int b = v & 1;
         ok = __all_sync(0xffffffffu, wait_b(&bar_sf[b], (v >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
         if (!ok) break;
@@ -407,9 +449,9 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
             sv[96 + e] = __uint_as_float(r3[e]);
           }
         }
-        if (vs[x].mask) {
-          const int cmin = max(0, dc - vs[x].hi);
-          const int cmax = min(BN - 1, dc - vs[x].lo);
+        if (vx.mask) {
+          const int cmin = max(0, dc - vx.hi);
+          const int cmax = min(BN - 1, dc - vx.lo);
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c < cmin || c > cmax) sv[c] = -INFINITY;
@@ -461,7 +503,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         tmem_wait_st();
         // the last visit: make sure PV_{v-1} is done so that exactly one PV
         // (this visit's) is outstanding when the epilogue waits
-        const bool last = (kt == t.qt) && (x == nv - 1);
+        const bool last = v == pl.n_all - 1;
         if (last && v > 0) {
           ok = __all_sync(0xffffffffu, wait_b(&bar_od, (v - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
         }
@@ -554,6 +596,407 @@ prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restric
   }
 }
 
+
+// ===========================================================================
+// Two heads per CTA.
+//
+// The CTA takes one 128-row query tile of two query heads of the same GQA
+// group: both read the same K/V tiles (loaded once), and two softmax
+// warpgroups ping-pong against one MMA warp, so the tensor core always has
+// the other head's QK or PV to run while a softmax warpgroup works.
+//   warps 0-3 / 4-7  softmax of head A / head B (thread = row = TMEM lane)
+//   warp 8           TMA producers: lane 0 streams Q and K tiles, lane 1 V tiles
+//   warp 9           TMEM allocator and tcgen05.mma issuer
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// Visit order: every grouped visit (ascending key tile), then every base
+// visit.  The query tiles are rotated in place into grouped positions for
+// the first phase and re-loaded by TMA for the second.
+// ===========================================================================
+constexpr int P2_THREADS = 320;
+constexpr int P2_NKS = 3;
+constexpr int P2_NVS = 2;
+constexpr int P2_OFF_Q = 0;                     // Q_A, Q_B: 2 x 32 KB
+constexpr int P2_OFF_K = 2 * TILE_BYTES;
+constexpr int P2_OFF_V = P2_OFF_K + P2_NKS * TILE_BYTES;
+constexpr int P2_SMEM_ALLOC = P2_OFF_V + P2_NVS * TILE_BYTES + 1024;
+
+__global__ void __launch_bounds__(P2_THREADS, 1)
+bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
+                        const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
+                        const __grid_constant__ Params p, const __grid_constant__ InvFreq inv) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_q, bar_qg[2], bar_qfree, bar_q2, bar_kf[P2_NKS], bar_ke[P2_NKS],
+      bar_vf[P2_NVS], bar_ve[P2_NVS], bar_sf[2], bar_pr[2], bar_od[2], bar_drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int s = blockIdx.z;
+  const int hA = 2 * blockIdx.y;  // heads hA, hA + 1 (same kv head: the group size is even)
+  const int a = p.cu[s];
+  const int L = p.cu[s + 1] - a;
+  if (L <= 0 || a < 0 || a + L > p.T) return;
+  const int nqt = (L + BM - 1) / BM;
+  if ((int)blockIdx.x >= nqt) return;
+  Tile t;
+  t.L = L;
+  t.qt = nqt - 1 - (int)blockIdx.x;
+  t.i0 = t.qt * BM;
+  t.i1 = min(t.i0 + BM - 1, L - 1);
+  t.G = p.plain ? 1 : (int)group_size(L, p.w_pre);
+  t.bif = t.G > 1;
+  const int kvh = hA / (p.Hq / p.Hkv);
+  // visits: grouped ones first
+  const VisitPlan pl = make_plan(t, p.w0);
+  const int n_grp = pl.n_grp, n_all = pl.n_all;
+  const bool reload_q = n_grp > 0 && n_all > n_grp;
+
+  const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
+  uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bar_q, 1);
+    mbar_init(&bar_qg[0], 128);
+    mbar_init(&bar_qg[1], 128);
+    mbar_init(&bar_qfree, 1);
+    mbar_init(&bar_q2, 1);
+    for (int i = 0; i < P2_NKS; ++i) { mbar_init(&bar_kf[i], 1); mbar_init(&bar_ke[i], 1); }
+    for (int i = 0; i < P2_NVS; ++i) { mbar_init(&bar_vf[i], 1); mbar_init(&bar_ve[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_sf[i], 1);
+      mbar_init(&bar_pr[i], 128);
+      mbar_init(&bar_od[i], 1);
+    }
+    mbar_init(&bar_drain, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (warp == 8 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mQ) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mK) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mV) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&mKg) : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  const int tok_q0 = a + t.i0;
+  if (warp == 8) {
+    // ================= producer: Q (twice if re-loaded), K tiles in visit order
+    if (lane == 0) {
+      mbar_expect_tx(&bar_q, 2 * TILE_BYTES);
+      for (int x = 0; x < 2; ++x) {
+        tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * TILE_BYTES, 0, hA + x, tok_q0);
+        tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * TILE_BYTES + HALF_BYTES, 64, hA + x, tok_q0);
+      }
+      bool ok = true, q2 = false;
+      int v = 0;
+      for (; ok && v < n_all;) {
+        int kt;
+        Visit vv;
+        visit_at(t, pl, p.w0, v, kt, vv);
+        if (!vv.grp && reload_q && !q2) {
+          // base phase: the grouped QKs are done with the rotated tiles
+          if (!(ok = wait_b(&bar_qfree, 0, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER))) break;
+          mbar_expect_tx(&bar_q2, 2 * TILE_BYTES);
+          for (int x = 0; x < 2; ++x) {
+            tma_load(&mQ, &bar_q2, sbase + P2_OFF_Q + x * TILE_BYTES, 0, hA + x, tok_q0);
+            tma_load(&mQ, &bar_q2, sbase + P2_OFF_Q + x * TILE_BYTES + HALF_BYTES, 64, hA + x, tok_q0);
+          }
+          q2 = true;
+        }
+        const int st = v % P2_NKS;
+        if (v >= P2_NKS && !(ok = wait_b(&bar_ke[st], ((v / P2_NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+          break;
+        const CUtensorMap *m = vv.grp ? &mKg : &mK;
+        const uint32_t dst = sbase + P2_OFF_K + st * TILE_BYTES;
+        mbar_expect_tx(&bar_kf[st], TILE_BYTES);
+        tma_load(m, &bar_kf[st], dst, 0, kvh, a + kt * BN);
+        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        ++v;
+      }
+      for (int u = max(0, v - P2_NKS); u < v; ++u)
+        wait_drain(&bar_kf[u % P2_NKS], (u / P2_NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
+      wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
+      if (q2) wait_drain(&bar_q2, 0, p.err, ERR_TIMEOUT_PRODUCER);
+    } else if (lane == 1) {
+      // ================= producer: V tiles in visit order
+      bool ok = true;
+      int v = 0;
+      for (; ok && v < n_all;) {
+        int kt;
+        Visit vv;
+        visit_at(t, pl, p.w0, v, kt, vv);
+        const int st = v % P2_NVS;
+        if (v >= P2_NVS && !(ok = wait_b(&bar_ve[st], ((v / P2_NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+          break;
+        const uint32_t dst = sbase + P2_OFF_V + st * TILE_BYTES;
+        mbar_expect_tx(&bar_vf[st], TILE_BYTES);
+        tma_load(&mV, &bar_vf[st], dst, 0, kvh, a + kt * BN);
+        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        ++v;
+      }
+      for (int u = max(0, v - P2_NVS); u < v; ++u)
+        wait_drain(&bar_vf[u % P2_NVS], (u / P2_NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
+    }
+  } else if (warp == 9) {
+    // ================= MMA issuer (one thread), fixed order:
+    //   QK_A(0) QK_B(0), then per visit v: PV_A(v) QK_A(v+1) PV_B(v) QK_B(v+1)
+    // so that each softmax warpgroup's next S is computed while the other
+    // head's PV runs.  S_x is reused by QK_x(v+1) only after PV_x(v) (which
+    // read P_x(v) from it) has been issued.
+    if (lane == 0) {
+      bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
+      if (ok && n_grp > 0)
+        ok = wait_b(&bar_qg[0], 0, &abort_flag, p.err, ERR_TIMEOUT_MMA) &&
+             wait_b(&bar_qg[1], 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
+      bool q2_seen = !reload_q;
+      auto issue_qk = [&](int x, int v) -> bool {
+        if (v >= n_grp && !q2_seen) {
+          // first base-phase QK: release the rotated query tiles, wait for
+          // the re-loaded ones
+          umma_commit(&bar_qfree);
+          if (!wait_b(&bar_q2, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+          q2_seen = true;
+        }
+        if (!wait_b(&bar_kf[v % P2_NKS], (v / P2_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t qaddr = sbase + P2_OFF_Q + x * TILE_BYTES;
+        const uint32_t kaddr = sbase + P2_OFF_K + (v % P2_NKS) * TILE_BYTES;
+        const uint32_t scol = tmem + (uint32_t)(x * 128);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_sf[x]);
+        if (x == 1) umma_commit(&bar_ke[v % P2_NKS]);  // both heads' QK issued
+        return true;
+      };
+      auto issue_pv = [&](int x, int v) -> bool {
+        if (!wait_b(&bar_pr[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        if (!wait_b(&bar_vf[v % P2_NVS], (v / P2_NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t vaddr = sbase + P2_OFF_V + (v % P2_NVS) * TILE_BYTES;
+        const uint32_t pcol = tmem + (uint32_t)(x * 128);
+        const uint32_t ocol = tmem + COL_O + (uint32_t)(x * 128);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV,
+                  (v > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&bar_od[x]);
+        if (x == 1) umma_commit(&bar_ve[v % P2_NVS]);
+        return true;
+      };
+      if (ok && n_all > 0) ok = issue_qk(0, 0) && issue_qk(1, 0);
+      for (int v = 0; ok && v < n_all; ++v) {
+        ok = issue_pv(0, v);
+        if (ok && v + 1 < n_all) ok = issue_qk(0, v + 1);
+        if (ok) ok = issue_pv(1, v);
+        if (ok && v + 1 < n_all) ok = issue_qk(1, v + 1);
+      }
+      umma_commit(&bar_drain);
+      wait_drain(&bar_drain, 0, p.err, ERR_TIMEOUT_MMA);
+    }
+  } else {
+    // ================= softmax warpgroups (warps 0-3: head A, 4-7: head B)
+    const int hx = warp >> 2;
+    const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t scol = tmem + lane_base + (uint32_t)(hx * 128);
+    const uint32_t ocol = tmem + lane_base + COL_O + (uint32_t)(hx * 128);
+    const int i = t.i0 + r;
+    const int h = hA + hx;
+    bool ok = true;
+    if (n_grp > 0) {
+      // rotate this head's query tile in place: Q_g = R(f(i) - i) Q~
+      ok = __all_sync(0xffffffffu, wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+      if (ok) {
+        uint8_t *qt = gbase + P2_OFF_Q + hx * TILE_BYTES;
+        for (int kk = 0; kk < 8; ++kk) {
+          const int u = r + 128 * kk;
+          const int row = u >> 3;
+          const int lc = (u & 7) ^ (row & 7);
+          const int n = corr_n(min(t.i0 + row, L - 1), t.G);
+          uint4 *qa = reinterpret_cast<uint4 *>(qt + u * 16);
+          uint4 *qb = reinterpret_cast<uint4 *>(qt + HALF_BYTES + u * 16);
+          uint4 xa = *qa, xb = *qb;
+          uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pa[e2]));
+            float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pb[e2]));
+            float c0, s0, c1, s1;
+            angle_cs(n, inv.v[lc * 8 + 2 * e2], c0, s0);
+            angle_cs(n, inv.v[lc * 8 + 2 * e2 + 1], c1, s1);
+            rot_back(fa.x, fb.x, c0, s0);
+            rot_back(fa.y, fb.y, c1, s1);
+            __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
+            __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
+            pa[e2] = *reinterpret_cast<uint32_t *>(&ra);
+            pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
+          }
+          *qa = xa;
+          *qb = xb;
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bar_qg[hx]);
+    }
+
+    float m_run = -INFINITY, l_run = 0.f;
+    int v = 0;
+    for (; ok && v < n_all;) {
+      int kt;
+      Visit vv;
+      visit_at(t, pl, p.w0, v, kt, vv);
+      ok = __all_sync(0xffffffffu, wait_b(&bar_sf[hx], v & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+      if (!ok) break;
+      tc_fence_after();
+      // columns c with distance dc - c outside [lo, hi] are masked; the
+      // visit-uniform mask flag selects a specialisation without compares
+      const int dc = i - kt * BN;
+      const int cmin = vv.mask ? max(0, dc - vv.hi) : 0;
+      const int cmax = vv.mask ? min(BN - 1, dc - vv.lo) : BN - 1;
+      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      auto visit_body = [&](auto masked) {
+        constexpr bool MASKED = decltype(masked)::value;
+        auto sel = [&](int c, uint32_t raw) -> float {
+          if constexpr (MASKED) return (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(raw);
+          else return __uint_as_float(raw);
+        };
+        // pass 1: row max; the four 32-column loads are in flight together
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        {
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          tmem_ld32(scol + 0, r0);
+          tmem_ld32(scol + 32, r1);
+          tmem_ld32(scol + 64, r2);
+          tmem_ld32(scol + 96, r3);
+          tmem_wait_ld_regs(r0);
+          tmem_wait_ld_regs(r1);
+          tmem_wait_ld_regs(r2);
+          tmem_wait_ld_regs(r3);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            m4[0] = fmaxf(m4[0], sel(e, r0[e]));
+            m4[1] = fmaxf(m4[1], sel(e + 32, r1[e]));
+            m4[2] = fmaxf(m4[2], sel(e + 64, r2[e]));
+            m4[3] = fmaxf(m4[3], sel(e + 96, r3[e]));
+          }
+        }
+        const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;
+        const float m_new = fmaxf(m_run, mt);
+        const bool need = (m_run != -INFINITY) && (m_new > m_run + 8.0f);
+        if (m_run == -INFINITY) m_run = m_new;
+        if (__any_sync(0xffffffffu, need)) {
+          // O_x holds PV of visits < v, all complete: QK_x(v) was issued after
+          // PV_x(v-1) and the S_x commit covers it
+          const float f = need ? ex2(m_run - m_new) : 1.0f;
+          if (need) {
+            l_run *= f;
+            m_run = m_new;
+          }
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint32_t rr[32];
+            tmem_ld32(ocol + c4 * 32, rr);
+            tmem_wait_ld_regs(rr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
+            tmem_st32(ocol + c4 * 32, rr);
+          }
+          tmem_wait_st();
+        }
+        // pass 2: P = exp2(s * scale - m) as bf16 pairs, 64 columns per round
+        // trip; chunk c4's 16 packed columns land on columns 16 c4 .. 16 c4 + 15,
+        // which have already been read
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(scol + h2 * 64, ra);
+          tmem_ld32(scol + h2 * 64 + 32, rb);
+          tmem_wait_ld_regs(ra);
+          tmem_wait_ld_regs(rb);
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const uint32_t(&rr)[32] = half ? rb : ra;
+            const int c0 = h2 * 64 + half * 32;
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = c0 + 2 * e;
+              const float x0 = sel(c, rr[2 * e]);
+              const float x1 = sel(c + 1, rr[2 * e + 1]);
+              const float p0 = ex2(fmaf(x0, p.sl2, -m_use));
+              const float p1 = ex2(fmaf(x1, p.sl2, -m_use));
+              l4[(e & 1) * 2] += p0;
+              l4[(e & 1) * 2 + 1] += p1;
+              __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+              pk[e] = *reinterpret_cast<uint32_t *>(&pb);
+            }
+            tmem_st16(scol + (c0 >> 1), pk);
+          }
+        }
+      };
+      if (vv.mask)
+        visit_body(std::true_type{});
+      else
+        visit_body(std::false_type{});
+      l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar_pr[hx]);
+      ++v;
+    }
+    // ---- epilogue: exactly one PV (the last) can be outstanding
+    if (ok && v > 0) ok = __all_sync(0xffffffffu, wait_b(&bar_od[hx], (v - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+      const bool row_ok = i < L;
+      __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * HD;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t rr[32];
+        tmem_ld32(ocol + c4 * 32, rr);
+        tmem_wait_ld_regs(rr);
+        if (row_ok) {
+#pragma unroll
+          for (int e8 = 0; e8 < 4; ++e8) {
+            uint4 o4;
+            uint32_t *po = reinterpret_cast<uint32_t *>(&o4);
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              __nv_bfloat162 ob = __floats2bfloat162_rn(__uint_as_float(rr[e8 * 8 + 2 * e2]) * inv_l,
+                                                        __uint_as_float(rr[e8 * 8 + 2 * e2 + 1]) * inv_l);
+              po[e2] = *reinterpret_cast<uint32_t *>(&ob);
+            }
+            *reinterpret_cast<uint4 *>(orow + c4 * 32 + e8 * 8) = o4;
+          }
+        }
+      }
+      if (row_ok && p.lse != nullptr)
+        p.lse[(size_t)h * p.T + tok_q0 + r] =
+            (l_run > 0.f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+  }
+}
+
 }  // namespace tc
 
 // ------------------------------------------------------------------ host
@@ -618,8 +1061,11 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
       return e;
     }
   }
-  e = cudaFuncSetAttribute(tc::bifocal_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           tc::SMEM_ALLOC);
+  const bool pair_heads = ((Hq / Hkv) % 2) == 0;  // two heads of one GQA group per CTA
+  e = pair_heads ? cudaFuncSetAttribute(tc::bifocal_prefill2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        tc::P2_SMEM_ALLOC)
+                 : cudaFuncSetAttribute(tc::bifocal_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        tc::SMEM_ALLOC);
   if (e != cudaSuccess) {
     *why = "smem attribute";
     return e;
@@ -637,8 +1083,13 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   p.lse = lse;
   p.err = err;
   p.sl2 = 1.4426950408889634f / sqrtf((float)tc::HD);
-  dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq, batch);
-  tc::bifocal_prefill_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
+  if (pair_heads) {
+    dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq / 2, batch);
+    tc::bifocal_prefill2_kernel<<<grid, tc::P2_THREADS, tc::P2_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
+  } else {
+    dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq, batch);
+    tc::bifocal_prefill_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) *why = "tensor-core prefill launch";
   return e;
