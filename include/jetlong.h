@@ -65,10 +65,6 @@ typedef enum {
                                      the comparison mode (G forced to 1)      */
 #define JL_FLAG_SIMT 0x2u         /* prefill: run the SIMT reference kernel
                                      instead of the tensor-core kernel       */
-#define JL_FLAG_PREROTATED_K 0x4u /* prefill: rotate K into grouped positions
-                                     once per key in a pre-pass instead of
-                                     per tile visit (ablation of the in-tile
-                                     correction rotation)                    */
 
 /* Human-readable name of a status code (static string). */
 const char *jl_status_string(jl_status s);

@@ -134,7 +134,7 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
   if ((s = check_heads(n_q_heads, n_kv_heads, head_dim)) != JL_OK) return s;
   if ((s = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return s;
   if (dtype != JL_BF16 && dtype != JL_FP32) return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-  if (flags & ~(uint32_t)(JL_FLAG_PLAIN_CAUSAL | JL_FLAG_SIMT | JL_FLAG_PREROTATED_K))
+  if (flags & ~(uint32_t)(JL_FLAG_PLAIN_CAUSAL | JL_FLAG_SIMT))
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (batch < 0 || total_tokens < 0 || max_seqlen < 0)
     return fail(JL_ERR_INVALID_ARG, "batch, total_tokens and max_seqlen must be >= 0");
@@ -152,8 +152,6 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
   cudaStream_t st = (cudaStream_t)stream;
   const bool use_simt = dtype == JL_FP32 || (flags & JL_FLAG_SIMT) || head_dim != 128;
   if (use_simt) {
-    if (flags & JL_FLAG_PREROTATED_K)
-      return fail(JL_ERR_INVALID_ARG, "JL_FLAG_PREROTATED_K applies to the tensor-core kernel only");
     cudaError_t e = jl::launch_simt_prefill(dtype == JL_BF16, head_dim, q, k, v, out, lse, cu_seqlens,
                                             batch, total_tokens, n_q_heads, n_kv_heads, w_pretrained,
                                             w0, inv, plain, st);

@@ -20,7 +20,6 @@ JL_OK, JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_CUDA, JL_ERR_WORKSPACE = r
 JL_BF16, JL_FP32 = 0, 1
 JL_FLAG_PLAIN_CAUSAL = 0x1
 JL_FLAG_SIMT = 0x2
-JL_FLAG_PREROTATED_K = 0x4
 
 _lib = None
 
