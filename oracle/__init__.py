@@ -16,6 +16,7 @@ from .bifocal import (  # noqa: F401
     rope_inv_freq,
     rope_rotate,
     bifocal_attention,
+    bifocal_attention_kv,
     bifocal_attention_ie_merge,
     bifocal_attention_from_raw,
     bifocal_decode,

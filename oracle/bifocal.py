@@ -220,6 +220,52 @@ def bifocal_attention(q, k, v, cu_seqlens, w_pretrained, w0, theta, rows=None, p
     return out, lse
 
 
+def bifocal_attention_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, w_pretrained, w0, theta, rows=None,
+                         plain=False, row_batch=64):
+    """Prefill of new tokens against keys that include an existing cache.
+
+    Sequence s has keys/values k, v[cu_k[s] : cu_k[s+1]] at positions
+    0 .. Lk-1 (standard RoPE, never rewritten) and Lq <= Lk queries
+    q[cu_q[s] : cu_q[s+1]] at the last positions Lk-Lq .. Lk-1.  G follows
+    the current length Lk (§1 "Agrupamento Dinâmico"; §2 "Rotação de Correção
+    On-the-Fly": generation streams across length boundaries without
+    rewriting the cache).  With Lq = Lk this is ``bifocal_attention``; with
+    Lq = 1 it is one ``bifocal_decode`` step.
+
+    Returns (out [len(rows), Hq, D], lse [Hq, len(rows)]) for the query rows
+    ``rows`` (global indices into q; default all).
+    """
+    Tq, Hq, D = q.shape
+    Hkv = k.shape[1]
+    group = Hq // Hkv
+    rows = np.arange(Tq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((len(rows), Hq, D))
+    lse = np.full((Hq, len(rows)), -np.inf)
+    for (aq, bq), (ak, bk) in zip(_seq_bounds(cu_seqlens_q), _seq_bounds(cu_seqlens_k)):
+        Lq, Lk = bq - aq, bk - ak
+        if Lq > Lk:
+            raise ValueError("a sequence has more queries than keys")
+        sel = np.nonzero((rows >= aq) & (rows < bq))[0]
+        if Lq == 0 or len(sel) == 0:
+            continue
+        G = group_size(Lk, w_pretrained)
+        offset = Lk - Lq
+        pos_j = np.arange(Lk, dtype=np.int64)
+        for kv in range(Hkv):
+            K = _take64(k, np.arange(ak, bk), kv)
+            V = _take64(v, np.arange(ak, bk), kv)
+            K_g = None if plain else rope_rotate(K, correction_shift(pos_j, G), theta)
+            for h in range(kv * group, (kv + 1) * group):
+                for c in range(0, len(sel), row_batch):
+                    idx = sel[c:c + row_batch]
+                    pos_i = offset + (rows[idx] - aq)
+                    o, l_ = _attend_rows_direct(_take64(q, rows[idx], h), pos_i, K, K_g, V, G, w0,
+                                                theta, plain)
+                    out[idx, h] = o
+                    lse[h, idx] = l_
+    return out, lse
+
+
 def bifocal_decode(q, k_cache, v_cache, seqlens, w_pretrained, w0, theta, plain=False):
     """One decode step, route A: the new query of sequence b sits at position
     L_b - 1 and attends to cache rows 0 .. L_b - 1 with G = G(L_b).

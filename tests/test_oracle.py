@@ -348,3 +348,59 @@ def test_planted_window_off_by_one_is_caught():
     bad, _ = oracle.bifocal_attention(qt, kt, v, [0, L], w_pre, w0 + 1, theta)
     assert np.max(np.abs(good[:, 0] - np.array(bo))) < 1e-11
     assert np.max(np.abs(bad[:, 0] - np.array(bo))) > 1e-6
+
+
+# --------------------------------------------------------------------------
+# Prefill of new tokens against an existing cache
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("L,n,D,w_pre,w0", [(23, 5, 8, 5, 7), (17, 17, 8, 4, 1), (30, 1, 4, 6, 0),
+                                            (40, 9, 8, 8, 40), (33, 12, 8, 11, 5)])
+def test_chunk_rows_match_pure_python_brute_force(L, n, D, w_pre, w0):
+    # queries are the last n positions of an L-token sequence; G = G(L)
+    theta = 1e4 if D == 8 else 500.0
+    q_raw, k_raw, v = _raw_case(L, 1, 1, D, seed=L * 13 + n)
+    qt, kt = _rotated(q_raw, k_raw, theta)
+    out, lse = oracle.bifocal_attention_kv(qt[L - n:], kt, v, [0, n], [0, L], w_pre, w0, theta)
+    bo, bl = oracle.brute_force_tiny(q_raw[:, 0].tolist(), k_raw[:, 0].tolist(), v[:, 0].tolist(),
+                                     w_pre, w0, theta)
+    assert np.max(np.abs(out[:, 0] - np.array(bo)[L - n:])) < 1e-11
+    assert np.max(np.abs(lse[0] - np.array(bl)[L - n:])) < 1e-11
+
+
+def test_chunks_of_a_growing_sequence_follow_the_current_length():
+    # three chunks appended to one sequence: each chunk's rows equal the full
+    # prefill of the prefix that ends with it (G of that prefix), batched varlen
+    D, theta, w_pre, w0 = 16, 1e4, 20, 6
+    q, k, v = _raw_case(70, 4, 2, D, seed=8)
+    bounds = [(0, 25), (25, 41), (41, 70)]
+    for a, b in bounds:
+        ref_o, ref_l = oracle.bifocal_attention(q[:b], k[:b], v[:b], [0, b], w_pre, w0, theta)
+        o, l_ = oracle.bifocal_attention_kv(q[a:b], k[:b], v[:b], [0, b - a], [0, b], w_pre, w0, theta)
+        assert np.max(np.abs(o - ref_o[a:b])) < 1e-13
+        assert np.max(np.abs(l_ - ref_l[:, a:b])) < 1e-13
+    # the same three chunks as one packed batch of three sequences
+    cu_q = np.array([0, 25, 41, 70])
+    kk = np.concatenate([k[:25], k[:41], k[:70]])
+    vv = np.concatenate([v[:25], v[:41], v[:70]])
+    cu_k = np.array([0, 25, 66, 136])
+    o, _ = oracle.bifocal_attention_kv(q, kk, vv, cu_q, cu_k, w_pre, w0, theta)
+    for (a, b) in bounds:
+        ref_o, _ = oracle.bifocal_attention(q[:b], k[:b], v[:b], [0, b], w_pre, w0, theta)
+        assert np.max(np.abs(o[a:b] - ref_o[a:b])) < 1e-13
+
+
+def test_one_query_chunk_is_a_decode_step():
+    D, theta, L = 16, 1e4, 90
+    q, k, v = _raw_case(L, 4, 2, D, seed=21)
+    o, l_ = oracle.bifocal_attention_kv(q[L - 1:], k, v, [0, 1], [0, L], 20, 7, theta)
+    do, dl = oracle.bifocal_decode(q[L - 1][None], k[None], v[None], [L], 20, 7, theta)
+    assert np.max(np.abs(o[0] - do[0])) < 1e-13
+    assert np.max(np.abs(l_[:, 0] - dl[0])) < 1e-13
+
+
+def test_chunk_rejects_more_queries_than_keys():
+    q, k, v = _raw_case(5, 1, 1, 4, seed=1)
+    with pytest.raises(ValueError):
+        oracle.bifocal_attention_kv(q, k[:3], v[:3], [0, 5], [0, 3], 4, 1, 1e4)
