@@ -87,7 +87,8 @@ jl_status jl_group_size(int64_t L, int64_t w_pretrained, int64_t *G_out);
 
 /*
  * jl_bifocal_prefill_workspace_size — bytes of device workspace that
- * jl_bifocal_prefill needs for these sizes and flags (0 if none).  The
+ * jl_bifocal_prefill needs for these sizes and flags (0 if none); for
+ * jl_bifocal_prefill_kv pass the key token count as total_tokens.  The
  * workspace must be 256-byte aligned; its contents need no initialisation and
  * are scratch between calls.
  */
@@ -130,6 +131,39 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v,
                              int32_t w0, double rope_theta, jl_dtype dtype,
                              uint32_t flags, void *workspace,
                              size_t workspace_bytes, void *stream);
+
+/*
+ * jl_bifocal_prefill_kv — prefill of new tokens against keys that include an
+ * existing cache (chunked prefill; §2 "Rotação de Correção On-the-Fly":
+ * generation streams across length boundaries and the cache of standard-RoPE
+ * keys is never rewritten).
+ *
+ * Sequence s has Lk = cu_seqlens_k[s+1] - cu_seqlens_k[s] keys and values
+ * (positions 0 .. Lk-1, rows cu_seqlens_k[s] .. of k and v) and
+ * Lq = cu_seqlens_q[s+1] - cu_seqlens_q[s] <= Lk queries, which are the
+ * newest tokens: positions Lk-Lq .. Lk-1.  G = G(Lk), the current length.
+ *   q, out      [total_q, Hq, D];  lse [Hq, total_q] fp32 or NULL
+ *   k, v        [total_k, Hkv, D]
+ *   cu_seqlens_q, cu_seqlens_k   device int32 [batch + 1], each starting at 0
+ *   max_seqlen_q >= every Lq
+ *   workspace   >= jl_bifocal_prefill_workspace_size(batch, total_k, ...)
+ * Other arguments as for jl_bifocal_prefill (which is this call with
+ * cu_seqlens_k = cu_seqlens_q).  Lq = 1 is one decode step.  The prefix
+ * sums live on the device and are not checked on the host: a sequence with
+ * Lq > Lk, or whose rows run past total_q / total_k, is skipped by the kernels
+ * and its rows of out and lse are left unwritten.
+ */
+jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v,
+                                void *out, float *lse,
+                                const int32_t *cu_seqlens_q,
+                                const int32_t *cu_seqlens_k, int32_t batch,
+                                int32_t total_q, int32_t total_k,
+                                int32_t max_seqlen_q, int32_t n_q_heads,
+                                int32_t n_kv_heads, int32_t head_dim,
+                                int64_t w_pretrained, int32_t w0,
+                                double rope_theta, jl_dtype dtype,
+                                uint32_t flags, void *workspace,
+                                size_t workspace_bytes, void *stream);
 
 /*
  * jl_bifocal_decode_workspace_size — bytes of device workspace for

@@ -140,3 +140,37 @@ def test_workspace_sizes_are_consistent():
     import torch
     assert jl.jl_bifocal_prefill_workspace_size(1, 1024, 2, 1, 64, torch.float32) == 0
     assert jl.jl_bifocal_prefill_workspace_size(1, 1024, 32, 8, 128, torch.bfloat16) >= 1024 * 8 * 128 * 2
+
+
+def _prefill_kv_raw(jl, **kw):
+    args = dict(q=1 << 12, k=1 << 12, v=1 << 12, out=1 << 12, lse=None, cuq=1 << 12, cuk=1 << 12, batch=1,
+                Tq=16, Tk=40, maxL=16, Hq=4, Hkv=2, D=128, w_pre=8, w0=4, theta=1e4, dtype=jl.JL_BF16,
+                flags=0, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    P = ctypes.c_void_p
+    return jl.lib().jl_bifocal_prefill_kv(
+        P(args["q"]), P(args["k"]), P(args["v"]), P(args["out"]), P(args["lse"]), P(args["cuq"]),
+        P(args["cuk"]), args["batch"], args["Tq"], args["Tk"], args["maxL"], args["Hq"], args["Hkv"],
+        args["D"], args["w_pre"], args["w0"], args["theta"], args["dtype"], args["flags"], P(args["ws"]),
+        args["ws_bytes"], P(args["stream"]))
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cuk=None), "JL_ERR_INVALID_ARG"),
+    (dict(cuq=None), "JL_ERR_INVALID_ARG"),
+    (dict(Tk=15), "JL_ERR_INVALID_ARG"),          # fewer keys than queries
+    (dict(Tk=-1), "JL_ERR_INVALID_ARG"),
+    (dict(maxL=17), "JL_ERR_INVALID_ARG"),
+    (dict(k=(1 << 12) + 8), "JL_ERR_INVALID_ARG"),
+    (dict(ws=None, ws_bytes=0), "JL_ERR_WORKSPACE"),  # sized by the key count
+])
+def test_prefill_kv_rejects_bad_arguments_before_launch(kw, status):
+    jl = _lib()
+    s = _prefill_kv_raw(jl, **kw)
+    assert jl.status_string(s) == status, jl.last_error()
+
+
+def test_prefill_kv_empty_queries_is_a_no_op():
+    jl = _lib()
+    assert _prefill_kv_raw(jl, Tq=0, maxL=0) == jl.JL_OK
+    assert _prefill_kv_raw(jl, batch=0) == jl.JL_OK

@@ -10,8 +10,9 @@
 
 namespace jl {
 cudaError_t launch_simt_prefill(bool bf16, int D, const void *q, const void *k, const void *v, void *out,
-                                float *lse, const int32_t *cu, int batch, int T_total, int Hq, int Hkv,
-                                long long w_pre, int w0, const InvFreq &inv, int plain, cudaStream_t st);
+                                float *lse, const int32_t *cu, const int32_t *cu_k, int batch, int T_total,
+                                int Tk, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv, int plain,
+                                cudaStream_t st);
 struct DecodePlan {
   int nsplit;
   int chunk;
@@ -25,9 +26,9 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
                           float *part_ml, int *err, void *out, float *lse, cudaStream_t st);
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags);
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
-                              const int32_t *cu, int batch, int T_total, int max_seqlen, int Hq,
-                              int Hkv, long long w_pre, int w0, const InvFreq &inv, int plain,
-                              uint32_t flags, void *ws, size_t ws_bytes, cudaStream_t st,
+                              const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
+                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv,
+                              int plain, uint32_t flags, void *ws, size_t ws_bytes, cudaStream_t st,
                               const char **why);
 }  // namespace jl
 
@@ -124,49 +125,64 @@ size_t jl_bifocal_prefill_workspace_size(int32_t batch, int32_t total_tokens, in
   return jl::tc_prefill_workspace(batch, total_tokens, n_q_heads, n_kv_heads, head_dim, flags);
 }
 
-jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
-                             const int32_t *cu_seqlens, int32_t batch, int32_t total_tokens,
-                             int32_t max_seqlen, int32_t n_q_heads, int32_t n_kv_heads,
-                             int32_t head_dim, int64_t w_pretrained, int32_t w0, double rope_theta,
-                             jl_dtype dtype, uint32_t flags, void *workspace,
-                             size_t workspace_bytes, void *stream) {
+jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, void *out, float *lse,
+                                const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t batch,
+                                int32_t total_q, int32_t total_k, int32_t max_seqlen_q, int32_t n_q_heads,
+                                int32_t n_kv_heads, int32_t head_dim, int64_t w_pretrained, int32_t w0,
+                                double rope_theta, jl_dtype dtype, uint32_t flags, void *workspace,
+                                size_t workspace_bytes, void *stream) {
   jl_status s;
   if ((s = check_heads(n_q_heads, n_kv_heads, head_dim)) != JL_OK) return s;
   if ((s = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return s;
   if (dtype != JL_BF16 && dtype != JL_FP32) return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   if (flags & ~(uint32_t)(JL_FLAG_PLAIN_CAUSAL | JL_FLAG_SIMT))
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
-  if (batch < 0 || total_tokens < 0 || max_seqlen < 0)
-    return fail(JL_ERR_INVALID_ARG, "batch, total_tokens and max_seqlen must be >= 0");
-  if (batch == 0 || total_tokens == 0) return ok();  // nothing to attend
-  if (cu_seqlens == nullptr) return fail(JL_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0)
+    return fail(JL_ERR_INVALID_ARG, "batch, token counts and max_seqlen must be >= 0");
+  if (batch == 0 || total_q == 0) return ok();  // nothing to attend
+  if (total_k < total_q)
+    return fail(JL_ERR_INVALID_ARG, "total_k (%d) < total_q (%d): every sequence needs Lq <= Lk", total_k, total_q);
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return fail(JL_ERR_INVALID_ARG, "cu_seqlens is NULL");
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr)
     return fail(JL_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || (lse && !aligned16(lse)))
     return fail(JL_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  if (max_seqlen == 0 || max_seqlen > total_tokens)
-    return fail(JL_ERR_INVALID_ARG, "max_seqlen must be in [1, total_tokens] (got %d)", max_seqlen);
+  if (max_seqlen_q == 0 || max_seqlen_q > total_q)
+    return fail(JL_ERR_INVALID_ARG, "max_seqlen must be in [1, total query tokens] (got %d)", max_seqlen_q);
 
   const jl::InvFreq inv = make_inv_freq(head_dim, rope_theta);
   const int plain = (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0;
   cudaStream_t st = (cudaStream_t)stream;
   const bool use_simt = dtype == JL_FP32 || (flags & JL_FLAG_SIMT) || head_dim != 128;
   if (use_simt) {
-    cudaError_t e = jl::launch_simt_prefill(dtype == JL_BF16, head_dim, q, k, v, out, lse, cu_seqlens,
-                                            batch, total_tokens, n_q_heads, n_kv_heads, w_pretrained,
-                                            w0, inv, plain, st);
+    cudaError_t e = jl::launch_simt_prefill(dtype == JL_BF16, head_dim, q, k, v, out, lse, cu_seqlens_q,
+                                            cu_seqlens_k, batch, total_q, total_k, n_q_heads, n_kv_heads,
+                                            w_pretrained, w0, inv, plain, st);
     return e == cudaSuccess ? ok() : cuda_fail(e, "SIMT prefill launch");
   }
-  const size_t need = jl::tc_prefill_workspace(batch, total_tokens, n_q_heads, n_kv_heads, head_dim, flags);
+  const size_t need = jl::tc_prefill_workspace(batch, total_k, n_q_heads, n_kv_heads, head_dim, flags);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need))
     return fail(JL_ERR_WORKSPACE, "prefill needs %zu workspace bytes (got %zu)", need, workspace_bytes);
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(JL_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   const char *why = nullptr;
-  cudaError_t e = jl::launch_tc_prefill(q, k, v, out, lse, cu_seqlens, batch, total_tokens, max_seqlen,
-                                        n_q_heads, n_kv_heads, w_pretrained, w0, inv, plain, flags,
+  cudaError_t e = jl::launch_tc_prefill(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
+                                        max_seqlen_q, n_q_heads, n_kv_heads, w_pretrained, w0, inv, plain, flags,
                                         workspace, workspace_bytes, st, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, why ? why : "tensor-core prefill launch");
+}
+
+jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
+                             const int32_t *cu_seqlens, int32_t batch, int32_t total_tokens,
+                             int32_t max_seqlen, int32_t n_q_heads, int32_t n_kv_heads,
+                             int32_t head_dim, int64_t w_pretrained, int32_t w0, double rope_theta,
+                             jl_dtype dtype, uint32_t flags, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+  // every token of every sequence is a query: the key prefix sums are the
+  // query prefix sums
+  return jl_bifocal_prefill_kv(q, k, v, out, lse, cu_seqlens, cu_seqlens, batch, total_tokens, total_tokens,
+                               max_seqlen, n_q_heads, n_kv_heads, head_dim, w_pretrained, w0, rope_theta, dtype,
+                               flags, workspace, workspace_bytes, stream);
 }
 
 size_t jl_bifocal_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,

@@ -63,8 +63,10 @@ constexpr int ERR_TIMEOUT_MMA = 2;
 constexpr int ERR_TIMEOUT_SOFTMAX = 4;
 
 struct Params {
-  const int32_t *cu;
+  const int32_t *cu;    // query prefix sums [batch + 1]
+  const int32_t *cu_k;  // key prefix sums [batch + 1]
   int batch, T, Hq, Hkv;
+  int Tk;               // key tokens
   long long w_pre;
   int w0, plain;
   __nv_bfloat16 *out;
@@ -162,17 +164,18 @@ constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) 
 constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 16);  // B (= V) is MN-major
 
 // --------------------------------------------------------- tile schedule
+// A query tile: rows i0..i1 of a sequence with L queries at positions
+// off + i (off = Lk - L) over keys 0..Lk-1; G follows Lk.
 struct Tile {
-  int L, G, i0, i1, qt, bif;
+  int L, G, i0, i1, qt, bif, Lk, off;
 };
 
 // Visits of a query tile, in order: the grouped visits (key tiles whose
-// pairs include a distance >= w0) on key tiles 0 .. kg_end-1, then the base
-// visits (pairs with distance < w0) on key tiles ks_begin .. qt.  A visit's
-// columns c with (i - j0 - c) outside [lo, hi] are masked when `mask` is set.
-// The diagonal tile is always masked: besides j > i it holds the keys at or
-// past L (zero-filled, or the next sequence's).  Everything is computed from
-// integers in registers (no per-visit arrays).
+// pairs include a distance >= w0) on key tiles 0 .. n_grp-1, then the base
+// visits (pairs with distance < w0) on key tiles ks_begin .. the last key
+// tile.  A visit's columns c with (p_i - j0 - c) outside [lo, hi] are masked
+// when `mask` is set.  Everything is computed from integers in registers (no
+// per-visit arrays).
 struct Visit {
   int grp, mask, lo, hi;
 };
@@ -183,22 +186,24 @@ struct VisitPlan {
 
 __device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
   VisitPlan pl;
+  const int pmin = t.off + t.i0, pmax = t.off + t.i1;  // row positions
+  const int kt_last = pmax / BN;                        // last key tile with a visible key
   if (!t.bif) {
     pl.n_grp = 0;
     pl.ks_begin = 0;
-    pl.n_all = t.qt + 1;
+    pl.n_all = kt_last + 1;
     return pl;
   }
-  // grouped: dmax(kt) = i1 - kt*BN >= w0
-  pl.n_grp = (t.i1 >= w0) ? min(t.qt, (t.i1 - w0) / BN) + 1 : 0;
-  // base: dmin(kt) <= w0 - 1; for kt < qt, dmin = i0 - kt*BN - (BN-1); the
-  // diagonal tile always qualifies when w0 >= 1
+  // grouped: dmax(kt) = pmax - kt*BN >= w0
+  pl.n_grp = (pmax >= w0) ? min(kt_last, (pmax - w0) / BN) + 1 : 0;
+  // base: dmin(kt) = pmin - (kt*BN + BN-1) <= w0 - 1; the last key tile always
+  // qualifies when w0 >= 1
   int nstd = 0;
-  pl.ks_begin = t.qt + 1;
+  pl.ks_begin = kt_last + 1;
   if (w0 > 0) {
-    const int x = t.i0 - (BN - 1) - (w0 - 1);  // need kt*BN >= x
-    pl.ks_begin = x <= 0 ? 0 : min(t.qt, (x + BN - 1) / BN);
-    nstd = t.qt - pl.ks_begin + 1;
+    const int x = pmin - (BN - 1) - (w0 - 1);  // need kt*BN >= x
+    pl.ks_begin = x <= 0 ? 0 : min(kt_last, (x + BN - 1) / BN);
+    nstd = kt_last - pl.ks_begin + 1;
   }
   pl.n_all = pl.n_grp + nstd;
   return pl;
@@ -208,15 +213,17 @@ __device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int
   const bool grp = v < pl.n_grp;
   kt = grp ? v : pl.ks_begin + (v - pl.n_grp);
   const int j0 = kt * BN;
-  const int j1 = min(j0 + BN - 1, t.L - 1);
-  const int dmin = t.i0 - j1, dmax = t.i1 - j0;
-  const int diag = kt == t.qt;
+  const int j1 = min(j0 + BN - 1, t.Lk - 1);
+  const int dmin = t.off + t.i0 - j1, dmax = t.off + t.i1 - j0;
+  // the tile holds a key past some row's position (this includes keys at or
+  // past Lk: zero-filled, or the next sequence's): the causal mask is needed
+  const int causal = j0 + BN - 1 > t.off + t.i0;
   if (grp) {
-    out = Visit{1, diag || dmin < w0, w0, HI_INF};
+    out = Visit{1, causal || dmin < w0, w0, HI_INF};
   } else if (!t.bif) {
-    out = Visit{0, diag, 0, HI_INF};
+    out = Visit{0, causal, 0, HI_INF};
   } else {
-    out = Visit{0, diag || dmax > w0 - 1, 0, w0 - 1};
+    out = Visit{0, causal || dmax > w0 - 1, 0, w0 - 1};
   }
 }
 
@@ -235,9 +242,11 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 
   // ---- work item (uniform across the CTA; invalid items exit before any barrier)
   const int s = blockIdx.z, h = blockIdx.y;
-  const int a = p.cu[s];
-  const int L = p.cu[s + 1] - a;
-  if (L <= 0 || a < 0 || a + L > p.T) return;
+  const int a = p.cu[s];                // first query token
+  const int L = p.cu[s + 1] - a;        // queries
+  const int ak = p.cu_k[s];             // first key token
+  const int Lk = p.cu_k[s + 1] - ak;    // keys: the sequence's current length
+  if (L <= 0 || a < 0 || a + L > p.T || Lk < L || ak < 0 || ak + Lk > p.Tk) return;
   const int nqt = (L + BM - 1) / BM;
   if ((int)blockIdx.x >= nqt) return;
   Tile t;
@@ -245,10 +254,12 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   t.qt = nqt - 1 - (int)blockIdx.x;  // heaviest query tiles launch first
   t.i0 = t.qt * BM;
   t.i1 = min(t.i0 + BM - 1, L - 1);
-  t.G = p.plain ? 1 : (int)group_size(L, p.w_pre);
+  t.Lk = Lk;
+  t.off = Lk - L;
+  t.G = p.plain ? 1 : (int)group_size(Lk, p.w_pre);
   t.bif = t.G > 1;
   const int kvh = h / (p.Hq / p.Hkv);
-  const bool need_qg = t.bif && t.i1 >= p.w0;
+  const bool need_qg = t.bif && t.off + t.i1 >= p.w0;
   const VisitPlan pl = make_plan(t, p.w0);
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
@@ -300,8 +311,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         const CUtensorMap *m = vx.grp ? &mKg : &mK;
         const uint32_t dst = sbase + OFF_K + st * TILE_BYTES;
         mbar_expect_tx(&bar_kf[st], TILE_BYTES);
-        tma_load(m, &bar_kf[st], dst, 0, kvh, a + kt * BN);
-        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        tma_load(m, &bar_kf[st], dst, 0, kvh, ak + kt * BN);
+        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
       }
       // drain: every load issued must land before the CTA may exit
       for (int u = max(0, v - NKS); u < v; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
@@ -321,8 +332,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
           break;
         const uint32_t dst = sbase + OFF_V + st * TILE_BYTES;
         mbar_expect_tx(&bar_vf[st], TILE_BYTES);
-        tma_load(&mV, &bar_vf[st], dst, 0, kvh, a + kt * BN);
-        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        tma_load(&mV, &bar_vf[st], dst, 0, kvh, ak + kt * BN);
+        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
       }
       for (int u = max(0, v - NVS); u < v; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
     }
@@ -391,7 +402,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
           const int u = r + 128 * kk;        // 16-byte chunk of the first half
           const int row = u >> 3;
           const int lc = (u & 7) ^ (row & 7);  // logical 8-column group
-          const int n = corr_n(min(t.i0 + row, L - 1), t.G);
+          const int n = corr_n(t.off + min(t.i0 + row, L - 1), t.G);
           uint4 xa = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + u * 16);
           uint4 xb = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + HALF_BYTES + u * 16);
           uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
@@ -423,7 +434,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       int kt;
       Visit vx;
       visit_at(t, pl, p.w0, v, kt, vx);
-      const int dc = i - kt * BN;  // column c has distance dc - c
+      const int dc = t.off + i - kt * BN;  // column c has distance dc - c
       {
         const int b = v & 1;
         ok = __all_sync(0xffffffffu, wait_b(&bar_sf[b], (v >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
@@ -633,9 +644,11 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.z;
   const int hA = 2 * blockIdx.y;  // heads hA, hA + 1 (same kv head: the group size is even)
-  const int a = p.cu[s];
-  const int L = p.cu[s + 1] - a;
-  if (L <= 0 || a < 0 || a + L > p.T) return;
+  const int a = p.cu[s];                // first query token
+  const int L = p.cu[s + 1] - a;        // queries
+  const int ak = p.cu_k[s];             // first key token
+  const int Lk = p.cu_k[s + 1] - ak;    // keys: the sequence's current length
+  if (L <= 0 || a < 0 || a + L > p.T || Lk < L || ak < 0 || ak + Lk > p.Tk) return;
   const int nqt = (L + BM - 1) / BM;
   if ((int)blockIdx.x >= nqt) return;
   Tile t;
@@ -643,7 +656,9 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   t.qt = nqt - 1 - (int)blockIdx.x;
   t.i0 = t.qt * BM;
   t.i1 = min(t.i0 + BM - 1, L - 1);
-  t.G = p.plain ? 1 : (int)group_size(L, p.w_pre);
+  t.Lk = Lk;
+  t.off = Lk - L;
+  t.G = p.plain ? 1 : (int)group_size(Lk, p.w_pre);
   t.bif = t.G > 1;
   const int kvh = hA / (p.Hq / p.Hkv);
   // visits: grouped ones first
@@ -717,8 +732,8 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         const CUtensorMap *m = vv.grp ? &mKg : &mK;
         const uint32_t dst = sbase + P2_OFF_K + st * TILE_BYTES;
         mbar_expect_tx(&bar_kf[st], TILE_BYTES);
-        tma_load(m, &bar_kf[st], dst, 0, kvh, a + kt * BN);
-        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        tma_load(m, &bar_kf[st], dst, 0, kvh, ak + kt * BN);
+        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
         ++v;
       }
       for (int u = max(0, v - P2_NKS); u < v; ++u)
@@ -738,8 +753,8 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
           break;
         const uint32_t dst = sbase + P2_OFF_V + st * TILE_BYTES;
         mbar_expect_tx(&bar_vf[st], TILE_BYTES);
-        tma_load(&mV, &bar_vf[st], dst, 0, kvh, a + kt * BN);
-        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, a + kt * BN);
+        tma_load(&mV, &bar_vf[st], dst, 0, kvh, ak + kt * BN);
+        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
         ++v;
       }
       for (int u = max(0, v - P2_NVS); u < v; ++u)
@@ -823,7 +838,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
           const int u = r + 128 * kk;
           const int row = u >> 3;
           const int lc = (u & 7) ^ (row & 7);
-          const int n = corr_n(min(t.i0 + row, L - 1), t.G);
+          const int n = corr_n(t.off + min(t.i0 + row, L - 1), t.G);
           uint4 *qa = reinterpret_cast<uint4 *>(qt + u * 16);
           uint4 *qb = reinterpret_cast<uint4 *>(qt + HALF_BYTES + u * 16);
           uint4 xa = *qa, xb = *qb;
@@ -861,7 +876,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       tc_fence_after();
       // columns c with distance dc - c outside [lo, hi] are masked; the
       // visit-uniform mask flag selects a specialisation without compares
-      const int dc = i - kt * BN;
+      const int dc = t.off + i - kt * BN;  // row position minus the tile's first key
       const int cmin = vv.mask ? max(0, dc - vv.hi) : 0;
       const int cmax = vv.mask ? min(BN - 1, dc - vv.lo) : BN - 1;
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1038,24 +1053,25 @@ size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint
 }
 
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
-                              const int32_t *cu, int batch, int T_total, int max_seqlen, int Hq, int Hkv,
-                              long long w_pre, int w0, const InvFreq &inv, int plain, uint32_t flags,
-                              void *ws, size_t ws_bytes, cudaStream_t st, const char **why) {
+                              const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
+                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv,
+                              int plain, uint32_t flags, void *ws, size_t ws_bytes, cudaStream_t st,
+                              const char **why) {
   (void)flags; (void)ws_bytes;
   int *err = reinterpret_cast<int *>(ws);
   __nv_bfloat16 *kg = reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(ws) + 256);
   CUtensorMap mQ, mK, mV, mKg;
-  if (!make_map(&mQ, q, T_total, Hq) || !make_map(&mK, k, T_total, Hkv) || !make_map(&mV, v, T_total, Hkv) ||
-      !make_map(&mKg, kg, T_total, Hkv)) {
+  if (!make_map(&mQ, q, T_total, Hq) || !make_map(&mK, k, Tk, Hkv) || !make_map(&mV, v, Tk, Hkv) ||
+      !make_map(&mKg, kg, Tk, Hkv)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
   if (!plain) {
-    const long long n = (long long)T_total * 8;
+    const long long n = (long long)Tk * 8;
     tc::prerotate_k_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        (const __nv_bfloat16 *)k, kg, cu, batch, T_total, Hkv, w_pre, inv);
+        (const __nv_bfloat16 *)k, kg, cu_k, batch, Tk, Hkv, w_pre, inv);
     if ((e = cudaGetLastError()) != cudaSuccess) {
       *why = "pre-rotation launch";
       return e;
@@ -1072,8 +1088,10 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   }
   tc::Params p;
   p.cu = cu;
+  p.cu_k = cu_k;
   p.batch = batch;
   p.T = T_total;
+  p.Tk = Tk;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.w_pre = w_pre;

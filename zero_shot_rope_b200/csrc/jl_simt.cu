@@ -20,8 +20,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128)
 simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     T *__restrict__ out, float *__restrict__ lse, const int32_t *__restrict__ cu,
-                    int batch, int T_total, int Hq, int Hkv, long long w_pre, int w0, InvFreq inv,
-                    int plain) {
+                    const int32_t *__restrict__ cu_k, int batch, int T_total, int Tk, int Hq, int Hkv,
+                    long long w_pre, int w0, InvFreq inv, int plain) {
   constexpr int NC = D / 32;
   constexpr int NP = NC / 2;  // rotation pairs per lane
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -37,10 +37,13 @@ simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     if (cu[mid] <= tok) lo = mid; else hi = mid;
   }
   const int a = cu[lo];
-  const int L = cu[lo + 1] - a;
-  const int i = tok - a;
-  if (a < 0 || L <= 0 || a + L > T_total || i < 0 || i >= L) return;  // inconsistent cu_seqlens
-  const int G = plain ? 1 : (int)group_size(L, w_pre);
+  const int L = cu[lo + 1] - a;  // queries of this sequence
+  const int ak = cu_k[lo];
+  const int Lk = cu_k[lo + 1] - ak;  // keys: the sequence's current length
+  if (a < 0 || L <= 0 || a + L > T_total || tok - a >= L || Lk < L || ak < 0 || ak + Lk > Tk)
+    return;  // inconsistent prefix sums
+  const int i = Lk - L + (tok - a);  // the query's position
+  const int G = plain ? 1 : (int)group_size(Lk, w_pre);
   const bool bif = G > 1;
   const int kvh = h / (Hq / Hkv);
   const float scale = rsqrtf((float)D);
@@ -63,7 +66,7 @@ simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
 #pragma unroll
   for (int c = 0; c < NC; ++c) acc[c] = 0.f;
   for (int j = 0; j <= i; ++j) {
-    const T *kp = k + ((size_t)(a + j) * Hkv + kvh) * D;
+    const T *kp = k + ((size_t)(ak + j) * Hkv + kvh) * D;
     float kx[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) kx[c] = to_f<T>(kp[lane + 32 * c]);
@@ -87,7 +90,7 @@ simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     const float corr = expf(m - m_new);
     const float p = expf(s - m_new);
     l = fmaf(l, corr, p);
-    const T *vp = v + ((size_t)(a + j) * Hkv + kvh) * D;
+    const T *vp = v + ((size_t)(ak + j) * Hkv + kvh) * D;
 #pragma unroll
     for (int c = 0; c < NC; ++c) acc[c] = fmaf(acc[c], corr, p * to_f<T>(vp[lane + 32 * c]));
     m = m_new;
@@ -99,16 +102,16 @@ simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
 }
 
 cudaError_t launch_simt_prefill(bool bf16, int D, const void *q, const void *k, const void *v, void *out,
-                                float *lse, const int32_t *cu, int batch, int T_total, int Hq, int Hkv,
-                                long long w_pre, int w0, const InvFreq &inv, int plain,
+                                float *lse, const int32_t *cu, const int32_t *cu_k, int batch, int T_total,
+                                int Tk, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv, int plain,
                                 cudaStream_t st) {
   const long long warps = (long long)T_total * Hq;
   if (warps == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((warps + 3) / 4);
 #define JL_SIMT(TT, DD)                                                                        \
   simt_prefill_kernel<TT, DD><<<blocks, 128, 0, st>>>((const TT *)q, (const TT *)k,            \
-                                                      (const TT *)v, (TT *)out, lse, cu, batch, \
-                                                      T_total, Hq, Hkv, w_pre, w0, inv, plain)
+                                                      (const TT *)v, (TT *)out, lse, cu, cu_k,  \
+                                                      batch, T_total, Tk, Hq, Hkv, w_pre, w0, inv, plain)
   if (bf16) {
     if (D == 128) JL_SIMT(__nv_bfloat16, 128);
     else if (D == 64) JL_SIMT(__nv_bfloat16, 64);

@@ -55,6 +55,9 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_prefill.restype = ctypes.c_int
     L.jl_bifocal_prefill.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32,
                                      c_i32, c_i64, c_i32, c_d, ctypes.c_int, c_u32, c_p, c_sz, c_p]
+    L.jl_bifocal_prefill_kv.restype = ctypes.c_int
+    L.jl_bifocal_prefill_kv.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32,
+                                        c_i32, c_i32, c_i64, c_i32, c_d, ctypes.c_int, c_u32, c_p, c_sz, c_p]
     L.jl_bifocal_decode_workspace_size.restype = c_sz
     L.jl_bifocal_decode_workspace_size.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32]
     L.jl_bifocal_decode.restype = ctypes.c_int
@@ -142,6 +145,29 @@ def jl_bifocal_prefill(q, k, v, cu_seqlens, max_seqlen, w_pretrained, w0, rope_t
                                     float(rope_theta), _dtype_code(q), int(flags), _ptr(ws),
                                     0 if ws is None else ws.numel() * ws.element_size(),
                                     _stream(stream)))
+    return out, lse
+
+
+def jl_bifocal_prefill_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, w_pretrained, w0, rope_theta,
+                          out=None, lse=None, flags=0, workspace=None, stream=None):
+    """Prefill of new tokens against keys that include an existing cache:
+    sequence s has its Lq queries at the last positions of its Lk keys.
+
+    q [Tq, Hq, D]; k, v [Tk, Hkv, D]; cu_seqlens_q / cu_seqlens_k int32 [B+1]
+    on the device.  Returns (out [Tq, Hq, D], lse [Hq, Tq] or None).
+    """
+    Tq, Hq, D = q.shape
+    Tk, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = jl_bifocal_prefill_workspace_size(B, Tk, Hq, Hkv, D, q.dtype, flags)
+    ws = _workspace(ws_bytes, q.device, workspace)
+    _check(lib().jl_bifocal_prefill_kv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                                       _ptr(cu_seqlens_k), B, Tq, Tk, int(max_seqlen_q), Hq, Hkv, D,
+                                       int(w_pretrained), int(w0), float(rope_theta), _dtype_code(q), int(flags),
+                                       _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                       _stream(stream)))
     return out, lse
 
 
