@@ -366,12 +366,13 @@ def run_ours(args, world, rank, local):
                    "decode_steps": n_dec, "decode_L": [wd.seqlens[0], wd.seqlens[0] + n_dec - 1],
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush needed)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": kernel_traffic("bifocal_prefill_kernel"),
-                     "kernel": "jl_bifocal_prefill (pre-rotation + tcgen05 attention kernel)",
+                     "frac": achieved / peak, "traffic": kernel_traffic("bifocal_prefill2_kernel"),
+                     "kernel": "jl_bifocal_prefill (K pre-rotation + bifocal_prefill2_kernel, two heads per CTA)",
                      "peak_kind": f"{peak_kind} bf16 sustained",
                      "frac_of_burst_peak": achieved / peaks["bf16_tflops"]},
         "decode": {"us_per_tok": dec_us_tok, "hbm_gbs": dec_gbs, "hbm_peak_gbs": peaks["hbm_gbs"],
                    "frac": dec_gbs / peaks["hbm_gbs"], "bytes_per_step": dec_bytes / n_dec,
+                   "traffic": kernel_traffic("decode_tc_kernel"),
                    "plain_us_per_tok": 1e3 * plain_dec_ms / n_dec,
                    "overhead_vs_plain": (statistics.mean(dec_ms) - plain_dec_ms) / plain_dec_ms},
         "prefill": {"ms": mean_pre_ms, "plain_ms": plain_pre_ms,
