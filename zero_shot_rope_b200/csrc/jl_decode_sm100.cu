@@ -15,8 +15,10 @@
 //              two 3-stage rings.
 //   warps 4-11 rotation warps: rotate the remote rows of each K tile in shared
 //              memory by R(delta_j - delta_i); thread t owns one 16-byte column
-//              chunk (8 pairs) of rows t/8 + 32m, so its angles advance by a
-//              fixed 32-key stride (fp32 cos/sin recurrence, fp64 seed).
+//              chunk (8 pairs) of rows t/8 + 32m.  The rotation of its first
+//              row advances once per tile (fp32 recurrence, fp64 seed); its
+//              other rows compose that with one of two tabulated offsets, so
+//              no row waits on another.  Two pairs per packed f32x2 op.
 //   warp 13    TMEM allocator and single-thread tcgen05.mma issuer, per tile
 //              S^T = K Q^T   (M = 128 keys, N = 16: the GQA heads, zero-padded)
 //              then O^T += V^T P  (M = 128 = head_dim, N = 16, V read MN-major)
@@ -106,6 +108,42 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// packed fp32 pairs: one instruction computes both lanes (sm_100 f32x2)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 f) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
 // byte offset of (row, 16-byte chunk) in a 16-row K-major SWIZZLE_128B operand
 // half (rows 128 B apart, chunk XOR-swizzled by row % 8)
 __device__ __forceinline__ int op_off(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
@@ -120,6 +158,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
   __shared__ float red[2][4][8];
+  // [entry][cos, sin][16-byte slot]: the 8 values of a chunk sit in slots
+  // 2 lc and 2 lc + 1, swapped for lc >= 4, so the 8 lanes of a phase (8
+  // distinct chunks) read 8 distinct bank groups
+  __shared__ float4 otab[8][2][16];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -259,27 +301,81 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     }
   } else if (warp >= 4) {
     // ======================= rotation warps =======================
+    // Thread t owns one 16-byte column chunk (8 pairs) of rows r0 + RS m of
+    // every tile.  Its row-r0 rotation (the tile base) advances once per tile;
+    // the other rows compose the base with a fixed offset rotation, so the
+    // rows of a tile do not wait on one another.  With J = j0 + r0 and
+    // rho = J mod G, the offset of row m is
+    //   n(J + RS m) - n(J) = RS m - floor(RS m / G) - [rho + (RS m mod G) >= G]
+    // and the base advances by TK - floor(TK / G) - [rho + (TK mod G) >= G]:
+    // each a choice between two increments, tabulated once per CTA.
+    static_assert(ROT_ROWS == 4, "offset table holds rows 1..3");
     constexpr int RS = TK / ROT_ROWS;  // row stride of one thread (32)
     const int t = threadIdx.x - 128;
     const int pc = t & 7;           // physical 16-byte chunk within a 128-byte row
     const int r0 = t >> 3;          // first row (0..RS-1); rows r0 + RS m
     const int lc = pc ^ (r0 & 7);   // logical chunk: pairs k = 8 lc .. 8 lc + 7
-    float ec[8], es[8], w1c[8], w1s[8], w0c[8], w0s[8];
-    int rm = 0;
-    const int stride_full = RS - RS / G;  // n(j + RS) - n(j) without a carry
-    const int smod = RS % G;
+    float bc[8], bs[8];             // rotation of row r0 of the current tile
+    int rho = 0, sm1 = 0, sm2 = 0, sm3 = 0, sb = 0;
     if (bif) {
+      if (t < 64) {
+        // offset table: entries 2(m-1) + carry for rows m = 1..3, 6 + carry
+        // for the base advance
+        const int tl = t & 7, en = t >> 3;
+        const int span = en < 6 ? RS * (en / 2 + 1) : TK;
+        const int d = span - span / G - (en & 1);
+        float c[8], sn[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) angle_cs(d, inv.v[tl * 8 + e], c[e], sn[e]);
+        const int sw = (tl >> 2) & 1;
+        otab[en][0][2 * tl + sw] = make_float4(c[0], c[1], c[2], c[3]);
+        otab[en][0][2 * tl + (sw ^ 1)] = make_float4(c[4], c[5], c[6], c[7]);
+        otab[en][1][2 * tl + sw] = make_float4(sn[0], sn[1], sn[2], sn[3]);
+        otab[en][1][2 * tl + (sw ^ 1)] = make_float4(sn[4], sn[5], sn[6], sn[7]);
+      }
       const int jf = kb + r0;
       const int ni = corr_n(i, G);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const double w = inv.v[lc * 8 + e];
-        angle_cs(corr_n(jf, G) - ni, w, ec[e], es[e]);
-        angle_cs(stride_full, w, w1c[e], w1s[e]);
-        angle_cs(stride_full - 1, w, w0c[e], w0s[e]);
-      }
-      rm = jf % G;
+      for (int e = 0; e < 8; ++e) angle_cs(corr_n(jf, G) - ni, inv.v[lc * 8 + e], bc[e], bs[e]);
+      rho = jf % G;
+      sm1 = RS % G;
+      sm2 = (2 * RS) % G;
+      sm3 = (3 * RS) % G;
+      sb = TK % G;
+      asm volatile("bar.sync 2, %0;" ::"n"(NROT * 32) : "memory");
     }
+    // (c, s) <- (c, s) x offset entry en of this thread's chunk
+    auto compose = [&](int en, float (&c)[8], float (&sn)[8]) {
+      const int sw = (lc >> 2) & 1;
+      const float4 c0 = otab[en][0][2 * lc + sw], c1 = otab[en][0][2 * lc + (sw ^ 1)];
+      const float4 s0 = otab[en][1][2 * lc + sw], s1 = otab[en][1][2 * lc + (sw ^ 1)];
+      const float2 oc[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
+                            make_float2(c1.z, c1.w)};
+      const float2 os[4] = {make_float2(s0.x, s0.y), make_float2(s0.z, s0.w), make_float2(s1.x, s1.y),
+                            make_float2(s1.z, s1.w)};
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        const float2 b_c = make_float2(bc[2 * e2], bc[2 * e2 + 1]);
+        const float2 b_s = make_float2(bs[2 * e2], bs[2 * e2 + 1]);
+        const float2 cc = sub2(mul2(b_c, oc[e2]), mul2(b_s, os[e2]));
+        const float2 ss = fma2(b_s, oc[e2], mul2(b_c, os[e2]));
+        c[2 * e2] = cc.x;
+        c[2 * e2 + 1] = cc.y;
+        sn[2 * e2] = ss.x;
+        sn[2 * e2 + 1] = ss.y;
+      }
+    };
+    auto advance_base = [&]() {
+      const int cy = rho + sb >= G ? 1 : 0;
+      float c[8], sn[8];
+      compose(6 + cy, c, sn);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        bc[e] = c[e];
+        bs[e] = sn[e];
+      }
+      rho += sb - cy * G;
+    };
     bool ok = true;
     for (int u = 0; u < ntiles && ok; ++u) {
       const int sk = u % NKS;
@@ -292,56 +388,38 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         for (int m = 0; m < ROT_ROWS; ++m) {
           const int r = r0 + RS * m;
           if (j0 + r < j_local) {
+            float rc[8], rs[8];
+            if (m == 0) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                rc[e] = bc[e];
+                rs[e] = bs[e];
+              }
+            } else {
+              const int smm = m == 1 ? sm1 : (m == 2 ? sm2 : sm3);
+              compose(2 * (m - 1) + (rho + smm >= G ? 1 : 0), rc, rs);
+            }
             uint4 *pa = reinterpret_cast<uint4 *>(kt + r * 128 + pc * 16);
             uint4 *pb = reinterpret_cast<uint4 *>(kt + HALF_BYTES + r * 128 + pc * 16);
             uint4 xa = *pa, xb = *pb;
             uint32_t *ua = reinterpret_cast<uint32_t *>(&xa), *ub = reinterpret_cast<uint32_t *>(&xb);
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
-              float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&ua[e2]));
-              float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&ub[e2]));
-              rot_back(fa.x, fb.x, ec[2 * e2], es[2 * e2]);
-              rot_back(fa.y, fb.y, ec[2 * e2 + 1], es[2 * e2 + 1]);
-              __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
-              __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
-              ua[e2] = *reinterpret_cast<uint32_t *>(&ra);
-              ub[e2] = *reinterpret_cast<uint32_t *>(&rb);
+              const float2 fa = bf2_to_f2(ua[e2]), fb = bf2_to_f2(ub[e2]);
+              const float2 cc = make_float2(rc[2 * e2], rc[2 * e2 + 1]);
+              const float2 ss = make_float2(rs[2 * e2], rs[2 * e2 + 1]);
+              ua[e2] = f2_to_bf2(fma2(fa, cc, mul2(fb, ss)));
+              ub[e2] = f2_to_bf2(sub2(mul2(fb, cc), mul2(fa, ss)));
             }
             *pa = xa;
             *pb = xb;
           }
-          // advance to key j + RS: n grows by RS - floor((j+RS)/G) + floor(j/G)
-          rm += smod;
-          const bool carry = rm >= G;
-          if (carry) rm -= G;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float wc = carry ? w0c[e] : w1c[e];
-            const float ws = carry ? w0s[e] : w1s[e];
-            const float c2 = ec[e] * wc - es[e] * ws;
-            const float s2 = es[e] * wc + ec[e] * ws;
-            ec[e] = c2;
-            es[e] = s2;
-          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        advance_base();
       } else if (bif) {
-        // no remote key in this tile: only advance the recurrence
-#pragma unroll 1
-        for (int m = 0; m < ROT_ROWS; ++m) {
-          rm += smod;
-          const bool carry = rm >= G;
-          if (carry) rm -= G;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float wc = carry ? w0c[e] : w1c[e];
-            const float ws = carry ? w0s[e] : w1s[e];
-            const float c2 = ec[e] * wc - es[e] * ws;
-            const float s2 = es[e] * wc + ec[e] * ws;
-            ec[e] = c2;
-            es[e] = s2;
-          }
-        }
+        // no remote key in this tile: only advance the base
+        advance_base();
       }
       mbar_arrive(&bar_kr[sk]);
     }
