@@ -106,3 +106,41 @@ def test_decode_ignores_garbage_past_the_length(D, dtype):
     ro, rl = oracle.bifocal_decode(q, kc, vc, [L], 300, 64, 1e6)
     assert_close(to_np(out), ro, dtype, "out")
     assert_close(to_np(lse), rl, dtype, "lse")
+
+
+def test_decode_replays_from_a_cuda_graph():
+    # The lengths live on the device and the split plan is sized by
+    # max_seqlen (here the cache capacity), so a captured step replays
+    # correctly after the caller updates q and seqlens in place, including
+    # steps where G changes.
+    J = jl()
+    dev = torch.device("cuda:0")
+    B, cap, Hq, Hkv, D, w_pre, w0 = 3, 3000, 16, 4, 128, 1000, 300
+    g = torch.Generator().manual_seed(77)
+    kc = torch.randn(B, cap, Hkv, D, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, cap, Hkv, D, generator=g).to(torch.bfloat16)
+    kcd, vcd = kc.to(dev), vc.to(dev)
+    q_st = torch.zeros(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    sl_st = torch.full((B,), 1, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q_st)
+    lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(J.jl_bifocal_decode_workspace_size(B, Hq, Hkv, D, cap), dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        J.jl_bifocal_decode(q_st, kcd, vcd, sl_st, cap, w_pre, w0, 1e6, out=out, lse=lse, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        J.jl_bifocal_decode(q_st, kcd, vcd, sl_st, cap, w_pre, w0, 1e6, out=out, lse=lse, workspace=ws)
+    for step, lens in enumerate(([999, 1000, 2000], [1000, 1001, 2001], [1, 2999, 3000])):
+        q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16)
+        q_st.copy_(q.to(dev))
+        sl_st.copy_(torch.tensor(lens, dtype=torch.int32).to(dev))
+        graph.replay()
+        torch.cuda.synchronize()
+        ro, rl = oracle.bifocal_decode(q, kc, vc, lens, w_pre, w0, 1e6)
+        assert_close(to_np(out), ro, torch.bfloat16, f"out step {step}")
+        assert_close(to_np(lse), rl, torch.bfloat16, f"lse step {step}")
+    assert int(ws[:4].view(torch.int32).item()) == 0
