@@ -20,7 +20,11 @@ Readings where the pages leave a step open (each also listed in the design doc):
 * RoPE is the half-split form: pair k is (x_k, x_{k+D/2}) and is rotated by the
   angle m * theta**(-2k/D);
 * scores are scaled by 1/sqrt(D); LSE is the natural log of the softmax
-  normaliser of the scaled scores.
+  normaliser of the scaled scores;
+* a sliding-window layer of a hybrid model (the pages: the method carries over
+  to hybrid attention stacks unchanged) masks keys with p_i - p_j >= window
+  (window keys including the query's own position, as for w0); the visible
+  keys follow the bifocal rule and G still follows the sequence length.
 
 Parity: pinned.  tests/test_oracle.py checks these functions against closed
 forms, invariants, the worked G examples, special cases that reduce to textbook
@@ -144,7 +148,7 @@ def _seq_bounds(cu_seqlens):
 # ---------------------------------------------------------------------------
 
 
-def _attend_rows_direct(q_rows, pos_i, K, K_g, V, G, w0, theta, plain):
+def _attend_rows_direct(q_rows, pos_i, K, K_g, V, G, w0, theta, plain, window=0):
     """Scores of query rows against keys 0..L-1 of one sequence and one head.
 
     q_rows [R, D] standard-RoPE queries at positions pos_i; K [L, D]
@@ -156,6 +160,9 @@ def _attend_rows_direct(q_rows, pos_i, K, K_g, V, G, w0, theta, plain):
       d >= w0  ->  s = <R(delta_i) Q~_i, R(delta_j) K~_j> / sqrt(D)  (remote, grouped)
     "Janela Local" / "Janela Remota" bullets of §1 and the correction rotation
     of §2.  ``plain`` scores every pair with the base RoPE (G irrelevant).
+    ``window`` > 0 is a sliding-window layer of a hybrid model ("Principais
+    Contribuições" 4 and the hybrid-architecture results): only keys with
+    d < window are visible, and the visible ones follow the rule above.
     """
     L, D = K.shape
     scale = 1.0 / math.sqrt(D)
@@ -168,7 +175,10 @@ def _attend_rows_direct(q_rows, pos_i, K, K_g, V, G, w0, theta, plain):
         q_g = rope_rotate(q_rows, correction_shift(pos_i, G), theta)
         S_grp = (q_g @ K_g.T) * scale
         S = np.where(dist < w0, S_std, S_grp)
-    S = np.where(dist >= 0, S, -np.inf)
+    visible = dist >= 0
+    if window > 0:
+        visible &= dist < window
+    S = np.where(visible, S, -np.inf)
     return _softmax_rows(S, V)
 
 
@@ -182,7 +192,7 @@ def _take64(t, idx, h):
 
 
 def bifocal_attention(q, k, v, cu_seqlens, w_pretrained, w0, theta, rows=None, plain=False,
-                      row_batch=64):
+                      row_batch=64, window=0):
     """Dynamic Bifocal RoPE causal GQA prefill attention, route A (direct).
 
     q [T, Hq, D], k/v [T, Hkv, D] (any float type, torch or numpy; computed in
@@ -190,6 +200,8 @@ def bifocal_attention(q, k, v, cu_seqlens, w_pretrained, w0, theta, rows=None, p
     h // (Hq / Hkv).
 
     ``rows``: optional sorted global token indices to evaluate (default: all).
+    ``window`` > 0: sliding-window layer (keys with p_i - p_j >= window are
+    masked; G still follows the sequence length).
     Returns (out [len(rows), Hq, D], lse [Hq, len(rows)]) in fp64.
     """
     T, Hq, D = q.shape
@@ -214,14 +226,14 @@ def bifocal_attention(q, k, v, cu_seqlens, w_pretrained, w0, theta, rows=None, p
                     idx = sel[c:c + row_batch]
                     pos_i = rows[idx] - a
                     o, l_ = _attend_rows_direct(_take64(q, rows[idx], h), pos_i, K, K_g, V, G, w0,
-                                                theta, plain)
+                                                theta, plain, window)
                     out[idx, h] = o
                     lse[h, idx] = l_
     return out, lse
 
 
 def bifocal_attention_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, w_pretrained, w0, theta, rows=None,
-                         plain=False, row_batch=64):
+                         plain=False, row_batch=64, window=0):
     """Prefill of new tokens against keys that include an existing cache.
 
     Sequence s has keys/values k, v[cu_k[s] : cu_k[s+1]] at positions
@@ -230,7 +242,8 @@ def bifocal_attention_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, w_pretrained, w0, 
     the current length Lk (§1 "Agrupamento Dinâmico"; §2 "Rotação de Correção
     On-the-Fly": generation streams across length boundaries without
     rewriting the cache).  With Lq = Lk this is ``bifocal_attention``; with
-    Lq = 1 it is one ``bifocal_decode`` step.
+    Lq = 1 it is one ``bifocal_decode`` step.  ``window`` as in
+    ``bifocal_attention``.
 
     Returns (out [len(rows), Hq, D], lse [Hq, len(rows)]) for the query rows
     ``rows`` (global indices into q; default all).
@@ -260,13 +273,13 @@ def bifocal_attention_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, w_pretrained, w0, 
                     idx = sel[c:c + row_batch]
                     pos_i = offset + (rows[idx] - aq)
                     o, l_ = _attend_rows_direct(_take64(q, rows[idx], h), pos_i, K, K_g, V, G, w0,
-                                                theta, plain)
+                                                theta, plain, window)
                     out[idx, h] = o
                     lse[h, idx] = l_
     return out, lse
 
 
-def bifocal_decode(q, k_cache, v_cache, seqlens, w_pretrained, w0, theta, plain=False):
+def bifocal_decode(q, k_cache, v_cache, seqlens, w_pretrained, w0, theta, plain=False, window=0):
     """One decode step, route A: the new query of sequence b sits at position
     L_b - 1 and attends to cache rows 0 .. L_b - 1 with G = G(L_b).
 
@@ -274,6 +287,7 @@ def bifocal_decode(q, k_cache, v_cache, seqlens, w_pretrained, w0, theta, plain=
     G is recomputed from the current length at every step.
 
     q [B, Hq, D]; k_cache, v_cache [B, Lcap, Hkv, D]; seqlens [B].
+    ``window`` as in ``bifocal_attention``.
     Returns (out [B, Hq, D], lse [B, Hq]).
     """
     q = _as64(q)
@@ -295,7 +309,8 @@ def bifocal_decode(q, k_cache, v_cache, seqlens, w_pretrained, w0, theta, plain=
             V = _as64(v_cache[b, :L, kv])
             K_g = None if plain else rope_rotate(K, correction_shift(pos_j, G), theta)
             for h in range(kv * group, (kv + 1) * group):
-                o, l_ = _attend_rows_direct(q[b, h][None, :], pos_i, K, K_g, V, G, w0, theta, plain)
+                o, l_ = _attend_rows_direct(q[b, h][None, :], pos_i, K, K_g, V, G, w0, theta, plain,
+                                            window)
                 out[b, h] = o[0]
                 lse[b, h] = l_[0]
     return out, lse
@@ -413,9 +428,11 @@ def bifocal_attention_from_raw(q_raw, k_raw, v, L, w_pretrained, w0, theta):
 # ---------------------------------------------------------------------------
 
 
-def causal_rope_attention(q, k, v):
+def causal_rope_attention(q, k, v, window=0):
     """Ordinary causal softmax attention of one sequence over already-rotated
-    q [L, Hq, D], k/v [L, Hkv, D], scale 1/sqrt(D).  Returns (out, lse)."""
+    q [L, Hq, D], k/v [L, Hkv, D], scale 1/sqrt(D).  ``window`` > 0 is the
+    textbook sliding window: query i sees keys i - window + 1 .. i.
+    Returns (out, lse)."""
     q, k, v = _as64(q), _as64(k), _as64(v)
     L, Hq, D = q.shape
     group = Hq // k.shape[1]
@@ -425,6 +442,8 @@ def causal_rope_attention(q, k, v):
         kv = h // group
         S = (q[:, h] @ k[:, kv].T) / math.sqrt(D)
         S[np.triu_indices(L, 1)] = -np.inf
+        if window > 0:
+            S[np.tril_indices(L, -window)] = -np.inf
         out[:, h], lse[h] = _softmax_rows(S, v[:, kv])
     return out, lse
 
@@ -434,13 +453,14 @@ def causal_rope_attention(q, k, v):
 # ---------------------------------------------------------------------------
 
 
-def brute_force_tiny(q_raw, k_raw, v, w_pretrained, w0, theta):
+def brute_force_tiny(q_raw, k_raw, v, w_pretrained, w0, theta, window=0):
     """Pure-Python double loop over (i, j) for one sequence and one head pair:
     q_raw [L][D], k_raw [L][D], v [L][D] as nested lists of floats.
 
     Each score rotates the raw vectors explicitly with math.cos / math.sin at
     the position the definition names (absolute inside the window, f(.)
     outside), builds the full L x L score table and normalises each row.
+    ``window`` > 0 keeps only the keys j > i - window.
     Returns (out [L][D], lse [L]).
     """
     L = len(q_raw)
@@ -459,8 +479,9 @@ def brute_force_tiny(q_raw, k_raw, v, w_pretrained, w0, theta):
 
     out, lse = [], []
     for i in range(L):
+        j_first = max(0, i - window + 1) if window > 0 else 0
         scores = []
-        for j in range(i + 1):
+        for j in range(j_first, i + 1):
             if i - j < w0:
                 a, b = rot(q_raw[i], i), rot(k_raw[j], j)
             else:
@@ -469,6 +490,6 @@ def brute_force_tiny(q_raw, k_raw, v, w_pretrained, w0, theta):
         m = max(scores)
         e = [math.exp(s - m) for s in scores]
         z = sum(e)
-        out.append([sum(e[j] * v[j][c] for j in range(i + 1)) / z for c in range(D)])
+        out.append([sum(e[j - j_first] * v[j][c] for j in range(j_first, i + 1)) / z for c in range(D)])
         lse.append(m + math.log(z))
     return out, lse

@@ -404,3 +404,80 @@ def test_chunk_rejects_more_queries_than_keys():
     q, k, v = _raw_case(5, 1, 1, 4, seed=1)
     with pytest.raises(ValueError):
         oracle.bifocal_attention_kv(q, k[:3], v[:3], [0, 5], [0, 3], 4, 1, 1e4)
+
+
+# --------------------------------------------------------------------------
+# Sliding-window layers of a hybrid model (keys with d >= window masked)
+# --------------------------------------------------------------------------
+
+
+WINDOWED = [  # (L, D, w_pretrained, w0, window)
+    (23, 8, 5, 7, 1), (23, 8, 5, 7, 2), (23, 8, 5, 7, 7), (23, 8, 5, 7, 8), (30, 4, 6, 0, 9),
+    (33, 8, 11, 5, 17), (17, 8, 4, 1, 16), (19, 8, 4, 3, 40), (40, 8, 8, 12, 25),
+]
+
+
+@pytest.mark.parametrize("L,D,w_pre,w0,window", WINDOWED)
+def test_window_rows_match_pure_python_brute_force(L, D, w_pre, w0, window):
+    theta = 1e4 if D == 8 else 500.0
+    q_raw, k_raw, v = _raw_case(L, 1, 1, D, seed=L * 7 + window)
+    qt, kt = _rotated(q_raw, k_raw, theta)
+    out, lse = oracle.bifocal_attention(qt, kt, v, [0, L], w_pre, w0, theta, window=window)
+    bo, bl = oracle.brute_force_tiny(q_raw[:, 0].tolist(), k_raw[:, 0].tolist(), v[:, 0].tolist(),
+                                     w_pre, w0, theta, window=window)
+    assert np.max(np.abs(out[:, 0] - np.array(bo))) < 1e-11
+    assert np.max(np.abs(lse[0] - np.array(bl))) < 1e-11
+
+
+@pytest.mark.parametrize("w_pre,w0,window", [(3, 10, 10), (5, 40, 7), (1, 16, 1), (7, 3, 3)])
+def test_window_not_wider_than_w0_is_textbook_sliding_window(w_pre, w0, window):
+    # every visible pair is local, so G plays no part
+    L, D, theta = 64, 16, 1e4
+    q, k, v = _raw_case(L, 4, 2, D, seed=window + w0)
+    out, lse = oracle.bifocal_attention(q, k, v, [0, L], w_pre, w0, theta, window=window)
+    ref_o, ref_l = oracle.causal_rope_attention(q, k, v, window=window)
+    assert np.max(np.abs(out - ref_o)) < 1e-13
+    assert np.max(np.abs(lse - ref_l)) < 1e-13
+
+
+def test_window_of_one_returns_each_value():
+    # closed form: each query sees only its own key (distance 0, local)
+    L, D = 40, 8
+    q, k, v = _raw_case(L, 2, 1, D, seed=5)
+    out, lse = oracle.bifocal_attention(q, k, v, [0, L], 4, 2, 1e4, window=1)
+    for h in range(2):
+        assert np.max(np.abs(out[:, h] - v[:, 0])) < 1e-14
+        own = np.einsum("id,id->i", q[:, h], k[:, 0]) / math.sqrt(D)
+        assert np.max(np.abs(lse[h] - own)) < 1e-13
+
+
+@pytest.mark.parametrize("window", [60, 61, 1000])
+def test_window_covering_the_sequence_changes_nothing(window):
+    L, D, theta = 60, 16, 1e4
+    q, k, v = _raw_case(L, 4, 1, D, seed=window)
+    a, la = oracle.bifocal_attention(q, k, v, [0, L], 16, 5, theta)
+    b, lb = oracle.bifocal_attention(q, k, v, [0, L], 16, 5, theta, window=window)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_windowed_decode_equals_last_prefill_row():
+    D, theta, L = 16, 1e4, 90
+    q, k, v = _raw_case(L, 4, 2, D, seed=31)
+    for window in (1, 5, 20, 33, 90):
+        po, pl = oracle.bifocal_attention(q, k, v, [0, L], 20, 7, theta, window=window)
+        do, dl = oracle.bifocal_decode(q[L - 1][None], k[None], v[None], [L], 20, 7, theta, window=window)
+        assert np.max(np.abs(po[L - 1] - do[0])) < 1e-13
+        assert np.max(np.abs(pl[:, L - 1] - dl[0])) < 1e-13
+
+
+def test_planted_sliding_window_off_by_one_is_caught():
+    # a window admitting one more key than asked must differ from the brute force
+    L, D, w_pre, w0, window, theta = 23, 8, 5, 3, 9, 1e4
+    q_raw, k_raw, v = _raw_case(L, 1, 1, D, seed=77)
+    qt, kt = _rotated(q_raw, k_raw, theta)
+    bo, _ = oracle.brute_force_tiny(q_raw[:, 0].tolist(), k_raw[:, 0].tolist(), v[:, 0].tolist(),
+                                    w_pre, w0, theta, window=window)
+    good, _ = oracle.bifocal_attention(qt, kt, v, [0, L], w_pre, w0, theta, window=window)
+    bad, _ = oracle.bifocal_attention(qt, kt, v, [0, L], w_pre, w0, theta, window=window + 1)
+    assert np.max(np.abs(good[:, 0] - np.array(bo))) < 1e-11
+    assert np.max(np.abs(bad[:, 0] - np.array(bo))) > 1e-6
