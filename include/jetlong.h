@@ -146,10 +146,17 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v,
  *   k, v        [total_k, Hkv, D]
  *   cu_seqlens_q, cu_seqlens_k   device int32 [batch + 1], each starting at 0
  *   max_seqlen_q >= every Lq
+ *   window      0 for a global attention layer; W >= 1 for a sliding-window
+ *               layer of a hybrid model ("Principais Contribuições" 4: the
+ *               method carries over to hybrid attention stacks unchanged):
+ *               keys at distance p_i - p_j >= W are hidden, the visible ones
+ *               follow the bifocal rule with G = G(Lk).  W <= w0 is plain
+ *               sliding-window RoPE attention.  Negative: JL_ERR_INVALID_ARG.
  *   workspace   >= jl_bifocal_prefill_workspace_size(batch, total_k, ...)
  * Other arguments as for jl_bifocal_prefill (which is this call with
- * cu_seqlens_k = cu_seqlens_q).  Lq = 1 is one decode step.  The prefix
- * sums live on the device and are not checked on the host: a sequence with
+ * cu_seqlens_k = cu_seqlens_q and window = 0).  Lq = 1 is one decode step.
+ * The prefix sums live on the device and are not checked on the host: a
+ * sequence with
  * Lq > Lk, or whose rows run past total_q / total_k, is skipped by the kernels
  * and its rows of out and lse are left unwritten.
  */
@@ -161,8 +168,9 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v,
                                 int32_t max_seqlen_q, int32_t n_q_heads,
                                 int32_t n_kv_heads, int32_t head_dim,
                                 int64_t w_pretrained, int32_t w0,
-                                double rope_theta, jl_dtype dtype,
-                                uint32_t flags, void *workspace,
+                                int32_t window, double rope_theta,
+                                jl_dtype dtype, uint32_t flags,
+                                void *workspace,
                                 size_t workspace_bytes, void *stream);
 
 /*
@@ -201,6 +209,27 @@ jl_status jl_bifocal_decode(const void *q, const void *k_cache,
                             double rope_theta, void *out, float *lse,
                             void *workspace, size_t workspace_bytes,
                             jl_dtype dtype, uint32_t flags, void *stream);
+
+/*
+ * jl_bifocal_decode_window — jl_bifocal_decode for a sliding-window layer of
+ * a hybrid model ("Principais Contribuições" 4: the method carries over to
+ * hybrid attention stacks unchanged).  The new query of sequence b attends to
+ * the keys max(0, L_b - window) .. L_b - 1 only, scored by the bifocal rule
+ * with G = G(L_b); window = 0 is jl_bifocal_decode.  The splits cover
+ * min(max_seqlen, window) keys, so a narrow window costs what its keys cost.
+ * All other arguments, the workspace size and the error behaviour are those
+ * of jl_bifocal_decode; a negative window is JL_ERR_INVALID_ARG.
+ */
+jl_status jl_bifocal_decode_window(const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *seqlens,
+                                   int32_t batch, int32_t cache_capacity,
+                                   int32_t max_seqlen, int32_t n_q_heads,
+                                   int32_t n_kv_heads, int32_t head_dim,
+                                   int64_t w_pretrained, int32_t w0,
+                                   int32_t window, double rope_theta,
+                                   void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, jl_dtype dtype,
+                                   uint32_t flags, void *stream);
 
 /*
  * jl_bifocal_decode_noalloc — jl_bifocal_decode without a caller workspace.

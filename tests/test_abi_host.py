@@ -144,15 +144,15 @@ def test_workspace_sizes_are_consistent():
 
 def _prefill_kv_raw(jl, **kw):
     args = dict(q=1 << 12, k=1 << 12, v=1 << 12, out=1 << 12, lse=None, cuq=1 << 12, cuk=1 << 12, batch=1,
-                Tq=16, Tk=40, maxL=16, Hq=4, Hkv=2, D=128, w_pre=8, w0=4, theta=1e4, dtype=jl.JL_BF16,
-                flags=0, ws=None, ws_bytes=0, stream=None)
+                Tq=16, Tk=40, maxL=16, Hq=4, Hkv=2, D=128, w_pre=8, w0=4, window=0, theta=1e4,
+                dtype=jl.JL_BF16, flags=0, ws=None, ws_bytes=0, stream=None)
     args.update(kw)
     P = ctypes.c_void_p
     return jl.lib().jl_bifocal_prefill_kv(
         P(args["q"]), P(args["k"]), P(args["v"]), P(args["out"]), P(args["lse"]), P(args["cuq"]),
         P(args["cuk"]), args["batch"], args["Tq"], args["Tk"], args["maxL"], args["Hq"], args["Hkv"],
-        args["D"], args["w_pre"], args["w0"], args["theta"], args["dtype"], args["flags"], P(args["ws"]),
-        args["ws_bytes"], P(args["stream"]))
+        args["D"], args["w_pre"], args["w0"], args["window"], args["theta"], args["dtype"], args["flags"],
+        P(args["ws"]), args["ws_bytes"], P(args["stream"]))
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -162,6 +162,7 @@ def _prefill_kv_raw(jl, **kw):
     (dict(Tk=-1), "JL_ERR_INVALID_ARG"),
     (dict(maxL=17), "JL_ERR_INVALID_ARG"),
     (dict(k=(1 << 12) + 8), "JL_ERR_INVALID_ARG"),
+    (dict(window=-1), "JL_ERR_INVALID_ARG"),
     (dict(ws=None, ws_bytes=0), "JL_ERR_WORKSPACE"),  # sized by the key count
 ])
 def test_prefill_kv_rejects_bad_arguments_before_launch(kw, status):
@@ -174,3 +175,31 @@ def test_prefill_kv_empty_queries_is_a_no_op():
     jl = _lib()
     assert _prefill_kv_raw(jl, Tq=0, maxL=0) == jl.JL_OK
     assert _prefill_kv_raw(jl, batch=0) == jl.JL_OK
+
+
+def test_decode_window_rejects_a_negative_window_and_validates_like_decode():
+    jl = _lib()
+    P = ctypes.c_void_p
+
+    def call(window, **kw):
+        a = dict(q=1 << 12, kc=1 << 12, vc=1 << 12, sl=1 << 12, ws=1 << 20, ws_bytes=1 << 30, D=128)
+        a.update(kw)
+        return jl.lib().jl_bifocal_decode_window(
+            P(a["q"]), P(a["kc"]), P(a["vc"]), P(a["sl"]), 1, 64, 64, 8, 2, a["D"], 16, 8, window, 1e6,
+            P(1 << 12), P(None), P(a["ws"]), a["ws_bytes"], jl.JL_BF16, 0, P(None))
+
+    assert jl.status_string(call(-1)) == "JL_ERR_INVALID_ARG"
+    assert jl.status_string(call(16, q=None)) == "JL_ERR_INVALID_ARG"
+    assert jl.status_string(call(16, D=80)) == "JL_ERR_UNSUPPORTED"
+    assert jl.status_string(call(16, ws=None)) == "JL_ERR_WORKSPACE"
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,D", [(1, 32, 8, 128), (3, 16, 4, 128), (64, 32, 8, 128), (2, 8, 8, 64)])
+def test_decode_workspace_covers_every_shorter_plan(B, Hq, Hkv, D):
+    # a sliding window plans its splits over fewer keys than max_seqlen: the
+    # workspace for max_seqlen must cover every such plan, i.e. be monotone
+    jl = _lib()
+    lens = sorted(set(list(range(1, 20000, 13)) + [2304, 2305, 131072]))
+    sizes = [jl.jl_bifocal_decode_workspace_size(B, Hq, Hkv, D, L) for L in lens]
+    assert all(x > 0 for x in sizes)
+    assert all(b >= a for a, b in zip(sizes, sizes[1:]))

@@ -11,8 +11,8 @@
 namespace jl {
 cudaError_t launch_simt_prefill(bool bf16, int D, const void *q, const void *k, const void *v, void *out,
                                 float *lse, const int32_t *cu, const int32_t *cu_k, int batch, int T_total,
-                                int Tk, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv, int plain,
-                                cudaStream_t st);
+                                int Tk, int Hq, int Hkv, long long w_pre, int w0, int window,
+                                const InvFreq &inv, int plain, cudaStream_t st);
 struct DecodePlan {
   int nsplit;
   int chunk;
@@ -22,14 +22,14 @@ DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int el
 size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen);
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
                           const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
-                          long long w_pre, int w0, const InvFreq &inv, int plain, float *part_o,
+                          long long w_pre, int w0, int window, const InvFreq &inv, int plain, float *part_o,
                           float *part_ml, int *err, void *out, float *lse, cudaStream_t st);
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags);
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
                               const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
-                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv,
-                              int plain, uint32_t flags, void *ws, size_t ws_bytes, cudaStream_t st,
-                              const char **why);
+                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, int window,
+                              const InvFreq &inv, int plain, uint32_t flags, void *ws, size_t ws_bytes,
+                              cudaStream_t st, const char **why);
 }  // namespace jl
 
 namespace {
@@ -129,11 +129,12 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
                                 const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int32_t batch,
                                 int32_t total_q, int32_t total_k, int32_t max_seqlen_q, int32_t n_q_heads,
                                 int32_t n_kv_heads, int32_t head_dim, int64_t w_pretrained, int32_t w0,
-                                double rope_theta, jl_dtype dtype, uint32_t flags, void *workspace,
-                                size_t workspace_bytes, void *stream) {
+                                int32_t window, double rope_theta, jl_dtype dtype, uint32_t flags,
+                                void *workspace, size_t workspace_bytes, void *stream) {
   jl_status s;
   if ((s = check_heads(n_q_heads, n_kv_heads, head_dim)) != JL_OK) return s;
   if ((s = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return s;
+  if (window < 0) return fail(JL_ERR_INVALID_ARG, "window must be >= 0 (0: no window), got %d", window);
   if (dtype != JL_BF16 && dtype != JL_FP32) return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   if (flags & ~(uint32_t)(JL_FLAG_PLAIN_CAUSAL | JL_FLAG_SIMT))
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
@@ -157,7 +158,7 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
   if (use_simt) {
     cudaError_t e = jl::launch_simt_prefill(dtype == JL_BF16, head_dim, q, k, v, out, lse, cu_seqlens_q,
                                             cu_seqlens_k, batch, total_q, total_k, n_q_heads, n_kv_heads,
-                                            w_pretrained, w0, inv, plain, st);
+                                            w_pretrained, w0, window, inv, plain, st);
     return e == cudaSuccess ? ok() : cuda_fail(e, "SIMT prefill launch");
   }
   const size_t need = jl::tc_prefill_workspace(batch, total_k, n_q_heads, n_kv_heads, head_dim, flags);
@@ -167,8 +168,8 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
     return fail(JL_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   const char *why = nullptr;
   cudaError_t e = jl::launch_tc_prefill(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
-                                        max_seqlen_q, n_q_heads, n_kv_heads, w_pretrained, w0, inv, plain, flags,
-                                        workspace, workspace_bytes, st, &why);
+                                        max_seqlen_q, n_q_heads, n_kv_heads, w_pretrained, w0, window, inv, plain,
+                                        flags, workspace, workspace_bytes, st, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, why ? why : "tensor-core prefill launch");
 }
 
@@ -181,8 +182,8 @@ jl_status jl_bifocal_prefill(const void *q, const void *k, const void *v, void *
   // every token of every sequence is a query: the key prefix sums are the
   // query prefix sums
   return jl_bifocal_prefill_kv(q, k, v, out, lse, cu_seqlens, cu_seqlens, batch, total_tokens, total_tokens,
-                               max_seqlen, n_q_heads, n_kv_heads, head_dim, w_pretrained, w0, rope_theta, dtype,
-                               flags, workspace, workspace_bytes, stream);
+                               max_seqlen, n_q_heads, n_kv_heads, head_dim, w_pretrained, w0, 0, rope_theta,
+                               dtype, flags, workspace, workspace_bytes, stream);
 }
 
 size_t jl_bifocal_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_t n_kv_heads,
@@ -194,13 +195,14 @@ size_t jl_bifocal_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_
   return 256 + align256(rows * head_dim * sizeof(float)) + align256(rows * 2 * sizeof(float));
 }
 
-jl_status jl_bifocal_decode(const void *q, const void *k_cache, const void *v_cache,
-                            const int32_t *seqlens, int32_t batch, int32_t cache_capacity,
-                            int32_t max_seqlen, int32_t n_q_heads, int32_t n_kv_heads,
-                            int32_t head_dim, int64_t w_pretrained, int32_t w0, double rope_theta,
-                            void *out, float *lse, void *workspace, size_t workspace_bytes,
-                            jl_dtype dtype, uint32_t flags, void *stream) {
+jl_status jl_bifocal_decode_window(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *seqlens, int32_t batch, int32_t cache_capacity,
+                                   int32_t max_seqlen, int32_t n_q_heads, int32_t n_kv_heads,
+                                   int32_t head_dim, int64_t w_pretrained, int32_t w0, int32_t window,
+                                   double rope_theta, void *out, float *lse, void *workspace,
+                                   size_t workspace_bytes, jl_dtype dtype, uint32_t flags, void *stream) {
   jl_status s;
+  if (window < 0) return fail(JL_ERR_INVALID_ARG, "window must be >= 0 (0: no window), got %d", window);
   if ((s = check_heads(n_q_heads, n_kv_heads, head_dim)) != JL_OK) return s;
   const int gs = n_q_heads / n_kv_heads;
   if (gs != 1 && gs != 2 && gs != 4 && gs != 8)
@@ -231,9 +233,20 @@ jl_status jl_bifocal_decode(const void *q, const void *k_cache, const void *v_ca
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e == cudaSuccess)
     e = jl::launch_decode(dtype == JL_BF16, head_dim, gs, q, k_cache, v_cache, seqlens, batch, cache_capacity,
-                          max_seqlen, n_q_heads, n_kv_heads, w_pretrained, w0, inv,
+                          max_seqlen, n_q_heads, n_kv_heads, w_pretrained, w0, window, inv,
                           (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0, part_o, part_ml, err, out, lse, st);
   return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
+}
+
+jl_status jl_bifocal_decode(const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *seqlens, int32_t batch, int32_t cache_capacity,
+                            int32_t max_seqlen, int32_t n_q_heads, int32_t n_kv_heads,
+                            int32_t head_dim, int64_t w_pretrained, int32_t w0, double rope_theta,
+                            void *out, float *lse, void *workspace, size_t workspace_bytes,
+                            jl_dtype dtype, uint32_t flags, void *stream) {
+  return jl_bifocal_decode_window(q, k_cache, v_cache, seqlens, batch, cache_capacity, max_seqlen, n_q_heads,
+                                  n_kv_heads, head_dim, w_pretrained, w0, 0, rope_theta, out, lse, workspace,
+                                  workspace_bytes, dtype, flags, stream);
 }
 
 }  // extern "C"

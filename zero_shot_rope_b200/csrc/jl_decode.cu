@@ -109,6 +109,7 @@ struct DecodeArgs {
   int Lcap, Hq, Hkv;
   long long w_pre;
   int w0, plain, chunk, nsplit;
+  int window;  // sliding-window width (0: none)
   float *part_o, *part_ml;
   int *err;
 };
@@ -131,10 +132,13 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap mK, const __grid_const
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, slot = tid / TPR, t = tid % TPR;
   int L = p.seqlens[b];
-  // a length outside [0, min(Lcap, nsplit * chunk)] attends to nothing rather
-  // than reading past the cache
-  if (L < 0 || L > p.Lcap || L > p.nsplit * p.chunk) L = 0;
-  const int kb = split * p.chunk;
+  // a length outside [0, Lcap], or with more keys than the planned splits
+  // hold, attends to nothing rather than reading past the cache; a
+  // sliding-window layer sees keys jw .. L-1 only
+  if (L < 0 || L > p.Lcap) L = 0;
+  int jw = p.window > 0 ? max(0, L - p.window) : 0;
+  if (L - jw > p.nsplit * p.chunk) L = jw = 0;
+  const int kb = jw + split * p.chunk;
   const int ke = min(L, kb + p.chunk);
   const int n = max(0, ke - kb);
   const size_t pidx = ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;  // + g * nsplit
@@ -454,22 +458,22 @@ static cudaError_t launch_decode_d(int GS, const CUtensorMap &mK, const CUtensor
 void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk);
 cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
                              const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                             const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o, float *part_ml,
-                             int *err, cudaStream_t st);
+                             int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
+                             float *part_ml, int *err, cudaStream_t st);
 
 static bool use_tc_decode(bool bf16, int D, int GS) { return bf16 && D == 128 && GS <= 8; }
 
-// Rows of split partials the workspace must hold: the largest of the plans
-// either decode kernel may use.
+// Rows of split partials the workspace must hold: a bound on the split count
+// of every plan either decode kernel may use for any key count up to
+// max_seqlen (a sliding window plans over fewer keys).  A plan never has more
+// splits than its per-(sequence, kv head) share of a wave, nor more than one
+// per key tile.
 size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
   const int GS = Hq / Hkv;
-  int ns = decode_plan(batch, Hq, Hkv, D, max_seqlen, 2).nsplit;
-  ns = max(ns, decode_plan(batch, Hq, Hkv, D, max_seqlen, 4).nsplit);
-  if (use_tc_decode(true, D, GS)) {
-    int nt, ct;
-    decode_tc_plan(batch, Hkv, max_seqlen, &nt, &ct);
-    ns = max(ns, nt);
-  }
+  const int per_bh = max(1, batch * Hkv);
+  const int tiles64 = (max(1, max_seqlen) + DEC_TK - 1) / DEC_TK;
+  int ns = min(max(1, 2 * 148 / per_bh), tiles64);  // both element sizes of decode_plan
+  if (use_tc_decode(true, D, GS)) ns = max(ns, min(max(1, 148 / per_bh), (max(1, max_seqlen) + 127) / 128));
   return (size_t)batch * Hq * ns;
 }
 
@@ -488,23 +492,25 @@ static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv) {
 
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
                           const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
-                          long long w_pre, int w0, const InvFreq &inv, int plain, float *part_o,
+                          long long w_pre, int w0, int window, const InvFreq &inv, int plain, float *part_o,
                           float *part_ml, int *err, void *out, float *lse, cudaStream_t st) {
   const int elem = bf16 ? 2 : 4;
+  // the splits cover at most `window` keys per sequence
+  const int keys = window > 0 ? min(max_seqlen, window) : max_seqlen;
   if (use_tc_decode(bf16, D, GS)) {
     CUtensorMap tK, tV;
     if (!make_tile_map(&tK, kc, B * Lcap, Hkv) || !make_tile_map(&tV, vc, B * Lcap, Hkv))
       return cudaErrorInvalidValue;
     int ns, chunk;
-    decode_tc_plan(B, Hkv, max_seqlen, &ns, &chunk);
+    decode_tc_plan(B, Hkv, keys, &ns, &chunk);
     cudaError_t e = launch_decode_tc(GS, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, Hq, Hkv, w_pre, w0,
-                                     inv, plain, ns, chunk, part_o, part_ml, err, st);
+                                     window, inv, plain, ns, chunk, part_o, part_ml, err, st);
     if (e != cudaSuccess) return e;
     decode_combine_kernel<__nv_bfloat16, 128><<<B * Hq, 128, 0, st>>>(part_o, part_ml, ns, (__nv_bfloat16 *)out,
                                                                       lse);
     return cudaGetLastError();
   }
-  const DecodePlan pl = decode_plan(B, Hq, Hkv, D, max_seqlen, elem);
+  const DecodePlan pl = decode_plan(B, Hq, Hkv, D, keys, elem);
   CUtensorMap mK, mV;
   if (!make_cache_map(&mK, kc, B * Lcap, Hkv, D, elem) || !make_cache_map(&mV, vc, B * Lcap, Hkv, D, elem))
     return cudaErrorInvalidValue;
@@ -517,6 +523,7 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
   a.w_pre = w_pre;
   a.w0 = w0;
   a.plain = plain;
+  a.window = window;
   a.chunk = pl.chunk;
   a.nsplit = pl.nsplit;
   a.part_o = part_o;

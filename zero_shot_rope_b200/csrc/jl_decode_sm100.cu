@@ -9,7 +9,7 @@
 // each remote key row is rotated once, by the relative shift, and the stored
 // query is used unchanged.
 //
-// CTA (split, kv head, sequence), 448 threads, keys [split*chunk, ...) in
+// CTA (split, kv head, sequence), 448 threads, keys [jw + split*chunk, ...) in
 // tiles of 128:
 //   warp 12    TMA producer: K and V tiles (128 keys x 128 d, SWIZZLE_128B) in
 //              two 3-stage rings.
@@ -68,6 +68,7 @@ struct Args {
   int Lcap, Hq, Hkv;
   long long w_pre;
   int w0, plain, chunk, nsplit;
+  int window;  // sliding-window width (0: none)
   float *part_o, *part_ml;
   int *err;
 };
@@ -166,8 +167,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   int L = p.seqlens[b];
-  if (L < 0 || L > p.Lcap || L > p.nsplit * p.chunk) L = 0;  // never read past the cache
-  const int kb = split * p.chunk;
+  if (L < 0 || L > p.Lcap) L = 0;  // never read past the cache
+  // a sliding-window layer sees keys jw .. L-1 only; the splits cover them
+  int jw = p.window > 0 ? max(0, L - p.window) : 0;
+  if (L - jw > p.nsplit * p.chunk) L = jw = 0;  // more keys than the planned splits hold
+  const int kb = jw + split * p.chunk;
   const int ke = min(L, kb + p.chunk);
   const int n = max(0, ke - kb);
   const size_t pidx = ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;  // + g * nsplit
@@ -607,8 +611,8 @@ void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk)
 
 cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
                              const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                             const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o, float *part_ml,
-                             int *err, cudaStream_t st) {
+                             int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
+                             float *part_ml, int *err, cudaStream_t st) {
   dtc::Args a;
   a.q = q;
   a.seqlens = seqlens;
@@ -618,6 +622,7 @@ cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &m
   a.w_pre = w_pre;
   a.w0 = w0;
   a.plain = plain;
+  a.window = window;
   a.chunk = chunk;
   a.nsplit = nsplit;
   a.part_o = part_o;

@@ -69,6 +69,7 @@ struct Params {
   int Tk;               // key tokens
   long long w_pre;
   int w0, plain;
+  int window;           // sliding-window width (0: none)
   __nv_bfloat16 *out;
   float *lse;
   int *err;
@@ -165,44 +166,54 @@ constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 16);  // B (= V) is MN-major
 
 // --------------------------------------------------------- tile schedule
 // A query tile: rows i0..i1 of a sequence with L queries at positions
-// off + i (off = Lk - L) over keys 0..Lk-1; G follows Lk.
+// off + i (off = Lk - L) over keys 0..Lk-1; G follows Lk.  W > 0 hides keys
+// at distance >= W (a sliding-window layer).
 struct Tile {
-  int L, G, i0, i1, qt, bif, Lk, off;
+  int L, G, i0, i1, qt, bif, Lk, off, W;
 };
 
 // Visits of a query tile, in order: the grouped visits (key tiles whose
-// pairs include a distance >= w0) on key tiles 0 .. n_grp-1, then the base
-// visits (pairs with distance < w0) on key tiles ks_begin .. the last key
-// tile.  A visit's columns c with (p_i - j0 - c) outside [lo, hi] are masked
-// when `mask` is set.  Everything is computed from integers in registers (no
-// per-visit arrays).
+// pairs include a distance in [w0, W)) on key tiles g_begin ..
+// g_begin + n_grp - 1, then the base visits (pairs with distance
+// < min(w0, W)) on key tiles ks_begin .. the last key tile.  A visit's
+// columns c with (p_i - j0 - c) outside [lo, hi] are masked when `mask` is
+// set.  Everything is computed from integers in registers (no per-visit
+// arrays).
 struct Visit {
   int grp, mask, lo, hi;
 };
 
 struct VisitPlan {
-  int n_grp, n_all, ks_begin;
+  int n_grp, n_all, ks_begin, g_begin;
 };
 
 __device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
   VisitPlan pl;
   const int pmin = t.off + t.i0, pmax = t.off + t.i1;  // row positions
   const int kt_last = pmax / BN;                        // last key tile with a visible key
+  // first key tile with a key inside the first row's window: dmin(kt) =
+  // pmin - (kt*BN + BN-1) <= W - 1
+  const int xw = pmin - t.W + 1;
+  const int kt_first = (t.W > 0 && xw > 0) ? xw / BN : 0;
+  pl.g_begin = kt_first;
   if (!t.bif) {
     pl.n_grp = 0;
-    pl.ks_begin = 0;
-    pl.n_all = kt_last + 1;
+    pl.ks_begin = kt_first;
+    pl.n_all = kt_last - kt_first + 1;
     return pl;
   }
-  // grouped: dmax(kt) = pmax - kt*BN >= w0
-  pl.n_grp = (pmax >= w0) ? min(kt_last, (pmax - w0) / BN) + 1 : 0;
-  // base: dmin(kt) = pmin - (kt*BN + BN-1) <= w0 - 1; the last key tile always
-  // qualifies when w0 >= 1
+  // grouped: dmax(kt) = pmax - kt*BN >= w0, and some grouped distance is
+  // inside the window
+  const bool any_grp = pmax >= w0 && (t.W == 0 || t.W > w0);
+  pl.n_grp = any_grp ? max(0, min(kt_last, (pmax - w0) / BN) - kt_first + 1) : 0;
+  // base: dmin(kt) = pmin - (kt*BN + BN-1) <= bl - 1 with bl = min(w0, W);
+  // the last key tile always qualifies when bl >= 1
+  const int bl = t.W > 0 ? min(w0, t.W) : w0;
   int nstd = 0;
   pl.ks_begin = kt_last + 1;
-  if (w0 > 0) {
-    const int x = pmin - (BN - 1) - (w0 - 1);  // need kt*BN >= x
-    pl.ks_begin = x <= 0 ? 0 : min(kt_last, (x + BN - 1) / BN);
+  if (bl > 0) {
+    const int x = pmin - (BN - 1) - (bl - 1);  // need kt*BN >= x
+    pl.ks_begin = max(kt_first, x <= 0 ? 0 : min(kt_last, (x + BN - 1) / BN));
     nstd = kt_last - pl.ks_begin + 1;
   }
   pl.n_all = pl.n_grp + nstd;
@@ -211,19 +222,21 @@ __device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
 
 __device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int w0, int v, int &kt, Visit &out) {
   const bool grp = v < pl.n_grp;
-  kt = grp ? v : pl.ks_begin + (v - pl.n_grp);
+  kt = grp ? pl.g_begin + v : pl.ks_begin + (v - pl.n_grp);
   const int j0 = kt * BN;
   const int j1 = min(j0 + BN - 1, t.Lk - 1);
   const int dmin = t.off + t.i0 - j1, dmax = t.off + t.i1 - j0;
   // the tile holds a key past some row's position (this includes keys at or
   // past Lk: zero-filled, or the next sequence's): the causal mask is needed
   const int causal = j0 + BN - 1 > t.off + t.i0;
+  const int whi = t.W > 0 ? t.W - 1 : HI_INF;  // largest visible distance
   if (grp) {
-    out = Visit{1, causal || dmin < w0, w0, HI_INF};
+    out = Visit{1, causal || dmin < w0 || dmax > whi, w0, whi};
   } else if (!t.bif) {
-    out = Visit{0, causal, 0, HI_INF};
+    out = Visit{0, causal || dmax > whi, 0, whi};
   } else {
-    out = Visit{0, causal || dmax > w0 - 1, 0, w0 - 1};
+    const int hi = min(w0 - 1, whi);
+    out = Visit{0, causal || dmax > hi, 0, hi};
   }
 }
 
@@ -256,11 +269,12 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   t.i1 = min(t.i0 + BM - 1, L - 1);
   t.Lk = Lk;
   t.off = Lk - L;
+  t.W = p.window;
   t.G = p.plain ? 1 : (int)group_size(Lk, p.w_pre);
   t.bif = t.G > 1;
   const int kvh = h / (p.Hq / p.Hkv);
-  const bool need_qg = t.bif && t.off + t.i1 >= p.w0;
   const VisitPlan pl = make_plan(t, p.w0);
+  const bool need_qg = pl.n_grp > 0;
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
@@ -658,6 +672,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   t.i1 = min(t.i0 + BM - 1, L - 1);
   t.Lk = Lk;
   t.off = Lk - L;
+  t.W = p.window;
   t.G = p.plain ? 1 : (int)group_size(Lk, p.w_pre);
   t.bif = t.G > 1;
   const int kvh = hA / (p.Hq / p.Hkv);
@@ -1054,9 +1069,9 @@ size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint
 
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
                               const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
-                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv,
-                              int plain, uint32_t flags, void *ws, size_t ws_bytes, cudaStream_t st,
-                              const char **why) {
+                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, int window,
+                              const InvFreq &inv, int plain, uint32_t flags, void *ws, size_t ws_bytes,
+                              cudaStream_t st, const char **why) {
   (void)flags; (void)ws_bytes;
   int *err = reinterpret_cast<int *>(ws);
   __nv_bfloat16 *kg = reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(ws) + 256);
@@ -1068,7 +1083,8 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   }
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
-  if (!plain) {
+  // grouped keys are needed unless the window keeps every visible pair local
+  if (!plain && !(window > 0 && window <= w0)) {
     const long long n = (long long)Tk * 8;
     tc::prerotate_k_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
         (const __nv_bfloat16 *)k, kg, cu_k, batch, Tk, Hkv, w_pre, inv);
@@ -1097,6 +1113,7 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   p.w_pre = w_pre;
   p.w0 = w0;
   p.plain = plain;
+  p.window = window;
   p.out = (__nv_bfloat16 *)out;
   p.lse = lse;
   p.err = err;

@@ -8,7 +8,8 @@
 // w0, otherwise the grouped score after the correction rotation of §2
 // "Rotação de Correção On-the-Fly" applied to the query and the key; the
 // single masked online softmax over those scores is the exact value of the
-// §2 inclusion–exclusion merge.
+// §2 inclusion–exclusion merge.  A sliding-window layer (window > 0) scores
+// only the keys at distance < window.
 //
 // Lane l holds elements l + 32c (c < D/32); the rotation pair of element
 // l + 32c (c < D/64) is element l + 32(c + D/64), so pairs never cross lanes.
@@ -21,7 +22,7 @@ __global__ void __launch_bounds__(128)
 simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     T *__restrict__ out, float *__restrict__ lse, const int32_t *__restrict__ cu,
                     const int32_t *__restrict__ cu_k, int batch, int T_total, int Tk, int Hq, int Hkv,
-                    long long w_pre, int w0, InvFreq inv, int plain) {
+                    long long w_pre, int w0, int window, InvFreq inv, int plain) {
   constexpr int NC = D / 32;
   constexpr int NP = NC / 2;  // rotation pairs per lane
   const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -65,7 +66,8 @@ simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
   float m = -INFINITY, l = 0.f, acc[NC];
 #pragma unroll
   for (int c = 0; c < NC; ++c) acc[c] = 0.f;
-  for (int j = 0; j <= i; ++j) {
+  // a sliding-window layer hides keys at distance >= window
+  for (int j = window > 0 ? max(0, i - window + 1) : 0; j <= i; ++j) {
     const T *kp = k + ((size_t)(ak + j) * Hkv + kvh) * D;
     float kx[NC];
 #pragma unroll
@@ -103,15 +105,15 @@ simt_prefill_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
 
 cudaError_t launch_simt_prefill(bool bf16, int D, const void *q, const void *k, const void *v, void *out,
                                 float *lse, const int32_t *cu, const int32_t *cu_k, int batch, int T_total,
-                                int Tk, int Hq, int Hkv, long long w_pre, int w0, const InvFreq &inv, int plain,
-                                cudaStream_t st) {
+                                int Tk, int Hq, int Hkv, long long w_pre, int w0, int window, const InvFreq &inv,
+                                int plain, cudaStream_t st) {
   const long long warps = (long long)T_total * Hq;
   if (warps == 0) return cudaSuccess;
   const unsigned blocks = (unsigned)((warps + 3) / 4);
 #define JL_SIMT(TT, DD)                                                                        \
   simt_prefill_kernel<TT, DD><<<blocks, 128, 0, st>>>((const TT *)q, (const TT *)k,            \
                                                       (const TT *)v, (TT *)out, lse, cu, cu_k,  \
-                                                      batch, T_total, Tk, Hq, Hkv, w_pre, w0, inv, plain)
+                                                      batch, T_total, Tk, Hq, Hkv, w_pre, w0, window, inv, plain)
   if (bf16) {
     if (D == 128) JL_SIMT(__nv_bfloat16, 128);
     else if (D == 64) JL_SIMT(__nv_bfloat16, 64);

@@ -57,12 +57,16 @@ def lib() -> ctypes.CDLL:
                                      c_i32, c_i64, c_i32, c_d, ctypes.c_int, c_u32, c_p, c_sz, c_p]
     L.jl_bifocal_prefill_kv.restype = ctypes.c_int
     L.jl_bifocal_prefill_kv.argtypes = [c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32,
-                                        c_i32, c_i32, c_i64, c_i32, c_d, ctypes.c_int, c_u32, c_p, c_sz, c_p]
+                                        c_i32, c_i32, c_i64, c_i32, c_i32, c_d, ctypes.c_int, c_u32, c_p, c_sz,
+                                        c_p]
     L.jl_bifocal_decode_workspace_size.restype = c_sz
     L.jl_bifocal_decode_workspace_size.argtypes = [c_i32, c_i32, c_i32, c_i32, c_i32]
     L.jl_bifocal_decode.restype = ctypes.c_int
     L.jl_bifocal_decode.argtypes = [c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64,
                                     c_i32, c_d, c_p, c_p, c_p, c_sz, ctypes.c_int, c_u32, c_p]
+    L.jl_bifocal_decode_window.restype = ctypes.c_int
+    L.jl_bifocal_decode_window.argtypes = [c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32, c_i64,
+                                           c_i32, c_i32, c_d, c_p, c_p, c_p, c_sz, ctypes.c_int, c_u32, c_p]
     L.jl_bifocal_decode_noalloc.restype = ctypes.c_int
     L.jl_bifocal_decode_noalloc.argtypes = [c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
                                             c_i64, c_i32, c_d, c_p, c_p, ctypes.c_int, c_u32, c_p]
@@ -149,9 +153,10 @@ def jl_bifocal_prefill(q, k, v, cu_seqlens, max_seqlen, w_pretrained, w0, rope_t
 
 
 def jl_bifocal_prefill_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, w_pretrained, w0, rope_theta,
-                          out=None, lse=None, flags=0, workspace=None, stream=None):
+                          out=None, lse=None, flags=0, workspace=None, stream=None, window=0):
     """Prefill of new tokens against keys that include an existing cache:
     sequence s has its Lq queries at the last positions of its Lk keys.
+    ``window`` > 0: sliding-window layer (keys at distance >= window hidden).
 
     q [Tq, Hq, D]; k, v [Tk, Hkv, D]; cu_seqlens_q / cu_seqlens_k int32 [B+1]
     on the device.  Returns (out [Tq, Hq, D], lse [Hq, Tq] or None).
@@ -165,7 +170,8 @@ def jl_bifocal_prefill_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, w_p
     ws = _workspace(ws_bytes, q.device, workspace)
     _check(lib().jl_bifocal_prefill_kv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
                                        _ptr(cu_seqlens_k), B, Tq, Tk, int(max_seqlen_q), Hq, Hkv, D,
-                                       int(w_pretrained), int(w0), float(rope_theta), _dtype_code(q), int(flags),
+                                       int(w_pretrained), int(w0), int(window), float(rope_theta), _dtype_code(q),
+                                       int(flags),
                                        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                                        _stream(stream)))
     return out, lse
@@ -186,6 +192,24 @@ def jl_bifocal_decode(q, k_cache, v_cache, seqlens, max_seqlen, w_pretrained, w0
                                    float(rope_theta), _ptr(out), _ptr(lse), _ptr(ws),
                                    0 if ws is None else ws.numel() * ws.element_size(),
                                    _dtype_code(q), int(flags), _stream(stream)))
+    return out, lse
+
+
+def jl_bifocal_decode_window(q, k_cache, v_cache, seqlens, max_seqlen, w_pretrained, w0, window, rope_theta,
+                             out=None, lse=None, flags=0, workspace=None, stream=None):
+    """jl_bifocal_decode for a sliding-window layer: the new query attends to
+    the last ``window`` keys of its sequence (0: all keys)."""
+    B, Hq, D = q.shape
+    Lcap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = jl_bifocal_decode_workspace_size(B, Hq, Hkv, D, int(max_seqlen))
+    ws = _workspace(ws_bytes, q.device, workspace)
+    _check(lib().jl_bifocal_decode_window(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), B, Lcap,
+                                          int(max_seqlen), Hq, Hkv, D, int(w_pretrained), int(w0), int(window),
+                                          float(rope_theta), _ptr(out), _ptr(lse), _ptr(ws),
+                                          0 if ws is None else ws.numel() * ws.element_size(),
+                                          _dtype_code(q), int(flags), _stream(stream)))
     return out, lse
 
 
