@@ -622,6 +622,24 @@ prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restric
 }
 
 
+// packed fp32 pairs (sm_100 f32x2): one instruction for two lanes of data
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // ===========================================================================
 // Two heads per CTA.
 //
@@ -894,7 +912,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       const int dc = t.off + i - kt * BN;  // row position minus the tile's first key
       const int cmin = vv.mask ? max(0, dc - vv.hi) : 0;
       const int cmax = vv.mask ? min(BN - 1, dc - vv.lo) : BN - 1;
-      float l4[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 l2a = make_float2(0.f, 0.f), l2b = make_float2(0.f, 0.f);
       auto visit_body = [&](auto masked) {
         constexpr bool MASKED = decltype(masked)::value;
         auto sel = [&](int c, uint32_t raw) -> float {
@@ -965,10 +983,11 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
               const int c = c0 + 2 * e;
               const float x0 = sel(c, rr[2 * e]);
               const float x1 = sel(c + 1, rr[2 * e + 1]);
-              const float p0 = ex2(fmaf(x0, p.sl2, -m_use));
-              const float p1 = ex2(fmaf(x1, p.sl2, -m_use));
-              l4[(e & 1) * 2] += p0;
-              l4[(e & 1) * 2 + 1] += p1;
+              const float2 a2 = ffma2(make_float2(x0, x1), make_float2(p.sl2, p.sl2), make_float2(-m_use, -m_use));
+              const float p0 = ex2(a2.x);
+              const float p1 = ex2(a2.y);
+              if (e & 1) l2b = fadd2(l2b, make_float2(p0, p1));
+              else l2a = fadd2(l2a, make_float2(p0, p1));
               __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
               pk[e] = *reinterpret_cast<uint32_t *>(&pb);
             }
@@ -980,7 +999,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         visit_body(std::true_type{});
       else
         visit_body(std::false_type{});
-      l_run += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      l_run += (l2a.x + l2a.y) + (l2b.x + l2b.y);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_pr[hx]);

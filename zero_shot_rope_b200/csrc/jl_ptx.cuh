@@ -62,9 +62,10 @@ __device__ __forceinline__ uint64_t gtime() {
   return t;
 }
 // Bounded wait: false on timeout (records `code`) or when another role aborted.
-static __device__ __noinline__ bool wait_b(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                    int *gerr, int code) {
-  if (mbar_try(bar, parity)) return true;
+// The first probe is inlined: most waits on the pipelines' critical paths find
+// the phase already complete, and a call there costs more than the probe.
+static __device__ __noinline__ bool wait_b_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                         int *gerr, int code) {
   const uint64_t t0 = gtime();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
@@ -77,6 +78,11 @@ static __device__ __noinline__ bool wait_b(uint64_t *bar, uint32_t parity, volat
       }
     }
   }
+}
+__device__ __forceinline__ bool wait_b(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *gerr,
+                                       int code) {
+  if (mbar_try(bar, parity)) return true;
+  return wait_b_slow(bar, parity, abort_flag, gerr, code);
 }
 // Bounded wait used only to let this CTA's own copies / MMAs land before it
 // exits; ignores the abort flag.
