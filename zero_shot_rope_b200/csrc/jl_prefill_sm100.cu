@@ -669,7 +669,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
                         const __grid_constant__ Params p, const __grid_constant__ InvFreq inv) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bar_q, bar_qg[2], bar_qfree, bar_q2, bar_kf[P2_NKS], bar_ke[P2_NKS],
-      bar_vf[P2_NVS], bar_ve[P2_NVS], bar_sf[2], bar_pr[2], bar_od[2], bar_drain;
+      bar_vf[P2_NVS], bar_ve[P2_NVS], bar_sf[2], bar_pr[2], bar_ph[2], bar_od[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
@@ -713,6 +713,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_sf[i], 1);
       mbar_init(&bar_pr[i], 128);
+      mbar_init(&bar_ph[i], 128);
       mbar_init(&bar_od[i], 1);
     }
     mbar_init(&bar_drain, 1);
@@ -828,16 +829,23 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         return true;
       };
       auto issue_pv = [&](int x, int v) -> bool {
-        if (!wait_b(&bar_pr[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        // P arrives in two halves (keys 0-63, then 64-127): the first half
+        // of PV runs while the softmax finishes the second
+        if (!wait_b(&bar_ph[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         if (!wait_b(&bar_vf[v % P2_NVS], (v / P2_NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
         const uint32_t vaddr = sbase + P2_OFF_V + (v % P2_NVS) * TILE_BYTES;
         const uint32_t pcol = tmem + (uint32_t)(x * 128);
         const uint32_t ocol = tmem + COL_O + (uint32_t)(x * 128);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
+        for (int kk = 0; kk < 4; ++kk)
           umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV,
                   (v > 0 || kk > 0) ? 1u : 0u);
+        if (!wait_b(&bar_pr[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 4; kk < 8; ++kk)
+          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV, 1u);
         umma_commit(&bar_od[x]);
         if (x == 1) umma_commit(&bar_ve[v % P2_NVS]);
         return true;
@@ -992,6 +1000,12 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
               pk[e] = *reinterpret_cast<uint32_t *>(&pb);
             }
             tmem_st16(scol + (c0 >> 1), pk);
+          }
+          if (h2 == 0) {
+            // keys 0-63 of P are in TMEM: the first half of PV may start
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar_ph[hx]);
           }
         }
       };
