@@ -358,6 +358,14 @@ def run_ours(args, world, rank, local):
         cpu = {"value": rows_flops(wp, rows) / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{len(rows)} random query rows x {wp.n_q_heads} heads of the {wp.seqlens[0]}-token "
                          f"prefill (fp64 NumPy oracle, {dt:.1f} s)"}
+        # the decode leg beside it: one full decode step (L = 131072) in the oracle
+        import oracle
+        L0 = int(wd.seqlens[0])
+        t0 = time.perf_counter()
+        oracle.bifocal_decode(qd_h[0], kc_h[:, :L0], vc_h[:, :L0], [L0], wd.w_pretrained, wd.w0, wd.rope_theta)
+        dt_d = time.perf_counter() - t0
+        cpu["decode"] = {"us_per_tok": dt_d * 1e6, "gbs": 2 * L0 * wd.n_kv_heads * wd.head_dim * 2 / dt_d / 1e9,
+                         "sample": f"one decode step at L = {L0} (fp64 NumPy oracle)"}
 
     if rank != 0:
         return

@@ -102,3 +102,47 @@ def test_full_size_workload_sampled_rows(name):
         far = rows[np.isin(rows, rows)]
         diff = np.abs(po - ro).mean()
         assert diff > 5 * err.mean(), (diff, err.mean())
+
+
+def test_planted_needles_peaked_attention():
+    # A key planted so that its score with one query is large under the
+    # method's own geometry (aligned with the query after the correction
+    # rotation for remote pairs, aligned as is inside the window) makes that
+    # row's attention peak on it: a wrong correction angle or a pair routed
+    # to the wrong branch moves most of the probability mass.  The plain
+    # causal oracle does not find the remote needles, so the rows also
+    # discriminate between the two modes.
+    L, Hq, Hkv, D, w_pre, w0, theta = 4096, 8, 2, 128, 1024, 256, 1e6   # G = 4
+    G = oracle.group_size(L, w_pre)
+    rng = np.random.default_rng(4242)
+    pos = np.arange(L)[:, None]
+    qt = oracle.rope_rotate(rng.standard_normal((L, Hq, D)), pos, theta)
+    kt = oracle.rope_rotate(rng.standard_normal((L, Hkv, D)), pos, theta)
+    v = rng.standard_normal((L, Hkv, D))
+    needles = []  # (row, distance)
+    for n, d in enumerate([300, 1000, 2500, 4000, 5, 200]):
+        i = L - 1 - 7 * n
+        j = i - d
+        for kv in range(Hkv):
+            qi = qt[i, kv * (Hq // Hkv)]
+            if d >= w0:   # grouped score <R(delta_i) q, R(delta_j) k> large
+                shift = oracle.correction_shift(i, G) - oracle.correction_shift(j, G)
+                kt[j, kv] = 1.5 * oracle.rope_rotate(qi, shift, theta)
+            else:
+                kt[j, kv] = 1.5 * qi
+            v[j, kv] = 4.0
+        needles.append((i, d))
+    q = torch.from_numpy(qt).to(torch.bfloat16)
+    k = torch.from_numpy(kt).to(torch.bfloat16)
+    vv = torch.from_numpy(v).to(torch.bfloat16)
+    cu = torch.tensor([0, L], dtype=torch.int32)
+    rows = np.array(sorted(i for i, _ in needles))
+    out, lse = prefill_gpu(q, k, vv, cu, w_pre, w0, theta)
+    ro, rl = oracle.bifocal_attention(q, k, vv, cu, w_pre, w0, theta, rows=rows)
+    assert_close(to_np(out)[rows], ro, torch.bfloat16, "needle rows")
+    assert_close(to_np(lse)[:, rows], rl, torch.bfloat16, "needle lse")
+    planted = [kv * (Hq // Hkv) for kv in range(Hkv)]
+    assert np.all(ro[:, planted, :].mean(axis=-1) > 3.9)   # the needle value is 4
+    po, _ = oracle.bifocal_attention(q, k, vv, cu, w_pre, w0, theta, rows=rows, plain=True)
+    remote = [n for n, r in enumerate(rows) if dict(needles)[r] >= w0]
+    assert po[remote][:, planted, :].mean() < 2.0
