@@ -146,3 +146,43 @@ def test_planted_needles_peaked_attention():
     po, _ = oracle.bifocal_attention(q, k, vv, cu, w_pre, w0, theta, rows=rows, plain=True)
     remote = [n for n, r in enumerate(rows) if dict(needles)[r] >= w0]
     assert po[remote][:, planted, :].mean() < 2.0
+
+
+D64_CASES = [
+    # (seqlens, Hq, Hkv, w_pre, w0) -- even GQA groups run the tensor-core kernel
+    ((100,), 4, 2, 40, 16),
+    ((129,), 2, 1, 64, 1),
+    ((777,), 8, 2, 160, 200),
+    ((1500,), 4, 2, 512, 0),
+    ((64, 0, 513, 1, 260), 8, 4, 128, 96),
+    ((1024,), 16, 8, 4096, 64),          # G = 1
+    ((600,), 4, 4, 100, 50),             # odd group: SIMT kernel
+]
+
+
+@pytest.mark.parametrize("seqlens,Hq,Hkv,w_pre,w0", D64_CASES)
+def test_head_dim_64_bf16_full(seqlens, Hq, Hkv, w_pre, w0):
+    q, k, v, cu = synth.random_case(sum(seqlens) + 64 + w0, seqlens, Hq, Hkv, 64, torch.bfloat16)
+    out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e4)
+    ro, rl = oracle.bifocal_attention(q, k, v, cu, w_pre, w0, 1e4)
+    assert_close(to_np(out), ro, torch.bfloat16, "out")
+    assert_close(to_np(lse), rl, torch.bfloat16, "lse")
+
+
+def test_head_dim_64_tensor_matches_simt_and_chunks():
+    J = jl()
+    q, k, v, cu = synth.random_case(17, (2000,), 8, 2, 64, torch.bfloat16)
+    a, _ = prefill_gpu(q, k, v, cu, 512, 300, 1e4)
+    b, _ = prefill_gpu(q, k, v, cu, 512, 300, 1e4, flags=J.JL_FLAG_SIMT)
+    err = (a.float() - b.float()).abs()
+    assert err.max().item() < 2e-2 and err.mean().item() < 2e-3
+    # a chunk of the last 700 tokens against the whole sequence, with a window
+    dev = torch.device("cuda:0")
+    cu_q = torch.tensor([0, 700], dtype=torch.int32)
+    o2, l2 = J.jl_bifocal_prefill_kv(q[1300:].contiguous().to(dev), k.to(dev), v.to(dev), cu_q.to(dev),
+                                     cu.to(dev), 700, 512, 300, 1e4, window=900,
+                                     lse=torch.empty(8, 700, device=dev))
+    torch.cuda.synchronize()
+    ro, rl = oracle.bifocal_attention_kv(q[1300:], k, v, cu_q, cu, 512, 300, 1e4, window=900)
+    assert_close(to_np(o2), ro, torch.bfloat16, "chunk out")
+    assert_close(to_np(l2), rl, torch.bfloat16, "chunk lse")

@@ -27,7 +27,7 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags);
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
                               const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
-                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, int window,
+                              int max_seqlen, int Hq, int Hkv, int D, long long w_pre, int w0, int window,
                               const InvFreq &inv, int plain, uint32_t flags, void *ws, size_t ws_bytes,
                               cudaStream_t st, const char **why);
 }  // namespace jl
@@ -121,7 +121,9 @@ size_t jl_bifocal_prefill_workspace_size(int32_t batch, int32_t total_tokens, in
                                          int32_t n_kv_heads, int32_t head_dim, jl_dtype dtype,
                                          uint32_t flags) {
   if (batch < 0 || total_tokens < 0 || n_q_heads <= 0 || n_kv_heads <= 0) return 0;
-  if (dtype != JL_BF16 || (flags & JL_FLAG_SIMT) || head_dim != 128) return 0;
+  if (n_q_heads % n_kv_heads != 0) return 0;
+  const bool tc_shape = head_dim == 128 || (head_dim == 64 && (n_q_heads / n_kv_heads) % 2 == 0);
+  if (dtype != JL_BF16 || (flags & JL_FLAG_SIMT) || !tc_shape) return 0;
   return jl::tc_prefill_workspace(batch, total_tokens, n_q_heads, n_kv_heads, head_dim, flags);
 }
 
@@ -154,7 +156,10 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
   const jl::InvFreq inv = make_inv_freq(head_dim, rope_theta);
   const int plain = (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0;
   cudaStream_t st = (cudaStream_t)stream;
-  const bool use_simt = dtype == JL_FP32 || (flags & JL_FLAG_SIMT) || head_dim != 128;
+  // tensor cores for bf16 at head_dim 128, and at 64 when the GQA group is
+  // even (the two-heads-per-CTA kernel); the SIMT kernel otherwise
+  const bool tc_shape = head_dim == 128 || (head_dim == 64 && (n_q_heads / n_kv_heads) % 2 == 0);
+  const bool use_simt = dtype == JL_FP32 || (flags & JL_FLAG_SIMT) || !tc_shape;
   if (use_simt) {
     cudaError_t e = jl::launch_simt_prefill(dtype == JL_BF16, head_dim, q, k, v, out, lse, cu_seqlens_q,
                                             cu_seqlens_k, batch, total_q, total_k, n_q_heads, n_kv_heads,
@@ -168,8 +173,8 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
     return fail(JL_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   const char *why = nullptr;
   cudaError_t e = jl::launch_tc_prefill(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, batch, total_q, total_k,
-                                        max_seqlen_q, n_q_heads, n_kv_heads, w_pretrained, w0, window, inv, plain,
-                                        flags, workspace, workspace_bytes, st, &why);
+                                        max_seqlen_q, n_q_heads, n_kv_heads, head_dim, w_pretrained, w0, window,
+                                        inv, plain, flags, workspace, workspace_bytes, st, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, why ? why : "tensor-core prefill launch");
 }
 

@@ -581,12 +581,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
 // Grouped keys K_g = R(f(j) - j) K~ for every token of sequences with G > 1,
 // written once per key (all kv heads of a token share the angles).
 __global__ void __launch_bounds__(256)
-prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kg,
+prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kg, int D,
                    const int32_t *__restrict__ cu, int batch, int T, int Hkv, long long w_pre,
                    const __grid_constant__ InvFreq inv) {
   const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gid >= (long long)T * 8) return;
-  const int tok = (int)(gid >> 3), cg = (int)(gid & 7);  // 8 pairs: k = 8cg .. 8cg+7
+  const int per_tok = D / 16;  // threads per token, 8 pairs each
+  if (gid >= (long long)T * per_tok) return;
+  const int tok = (int)(gid / per_tok), cg = (int)(gid % per_tok);  // pairs k = 8cg .. 8cg+7
   int lo = 0, hi = batch;
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -601,9 +602,9 @@ prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restric
 #pragma unroll
   for (int e = 0; e < 8; ++e) angle_cs(n, inv.v[cg * 8 + e], cs[e], sn[e]);
   for (int hh = 0; hh < Hkv; ++hh) {
-    const size_t base = ((size_t)tok * Hkv + hh) * HD + cg * 8;
+    const size_t base = ((size_t)tok * Hkv + hh) * D + cg * 8;
     uint4 xa = *reinterpret_cast<const uint4 *>(k + base);
-    uint4 xb = *reinterpret_cast<const uint4 *>(k + base + HD / 2);
+    uint4 xb = *reinterpret_cast<const uint4 *>(k + base + D / 2);
     uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
 #pragma unroll
     for (int e2 = 0; e2 < 4; ++e2) {
@@ -617,7 +618,7 @@ prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restric
       pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
     }
     *reinterpret_cast<uint4 *>(kg + base) = xa;
-    *reinterpret_cast<uint4 *>(kg + base + HD / 2) = xb;
+    *reinterpret_cast<uint4 *>(kg + base + D / 2) = xb;
   }
 }
 
@@ -658,11 +659,25 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 constexpr int P2_THREADS = 320;
 constexpr int P2_NKS = 3;
 constexpr int P2_NVS = 2;
-constexpr int P2_OFF_Q = 0;                     // Q_A, Q_B: 2 x 32 KB
-constexpr int P2_OFF_K = 2 * TILE_BYTES;
-constexpr int P2_OFF_V = P2_OFF_K + P2_NKS * TILE_BYTES;
-constexpr int P2_SMEM_ALLOC = P2_OFF_V + P2_NVS * TILE_BYTES + 1024;
+constexpr int P2_OFF_Q = 0;  // Q_A, Q_B
 
+// Tile geometry for a head_dim D (64 or 128): a tile row of D bf16 is D / 64
+// SWIZZLE_128B boxes of 64 columns (HALF_BYTES each for 128 rows).  O_x sits
+// at TMEM columns COL_O + x * D.
+template <int D>
+struct Geo {
+  static constexpr int NH = D / 64;          // 64-column boxes per tile row
+  static constexpr int TB = BM * D * 2;      // one Q, K or V tile
+  static constexpr int KSTEPS = D / 16;      // k-steps of a QK product
+  static constexpr int OFF_K = P2_OFF_Q + 2 * TB;
+  static constexpr int OFF_V = OFF_K + P2_NKS * TB;
+  static constexpr int SMEM_ALLOC = OFF_V + P2_NVS * TB + 1024;
+  // kind::f16, D fp32, A/B bf16, M = 128, N = D, B (= V) MN-major
+  static constexpr uint32_t IDESC_PV =
+      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((128u >> 4) << 24);
+};
+
+template <int D>
 __global__ void __launch_bounds__(P2_THREADS, 1)
 bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                         const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
@@ -673,6 +688,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
 
+  using GG = Geo<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.z;
   const int hA = 2 * blockIdx.y;  // heads hA, hA + 1 (same kv head: the group size is even)
@@ -739,11 +755,10 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   if (warp == 8) {
     // ================= producer: Q (twice if re-loaded), K tiles in visit order
     if (lane == 0) {
-      mbar_expect_tx(&bar_q, 2 * TILE_BYTES);
-      for (int x = 0; x < 2; ++x) {
-        tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * TILE_BYTES, 0, hA + x, tok_q0);
-        tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * TILE_BYTES + HALF_BYTES, 64, hA + x, tok_q0);
-      }
+      mbar_expect_tx(&bar_q, 2 * GG::TB);
+      for (int x = 0; x < 2; ++x)
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * GG::TB + hf * HALF_BYTES, 64 * hf, hA + x, tok_q0);
       bool ok = true, q2 = false;
       int v = 0;
       for (; ok && v < n_all;) {
@@ -753,21 +768,20 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         if (!vv.grp && reload_q && !q2) {
           // base phase: the grouped QKs are done with the rotated tiles
           if (!(ok = wait_b(&bar_qfree, 0, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER))) break;
-          mbar_expect_tx(&bar_q2, 2 * TILE_BYTES);
-          for (int x = 0; x < 2; ++x) {
-            tma_load(&mQ, &bar_q2, sbase + P2_OFF_Q + x * TILE_BYTES, 0, hA + x, tok_q0);
-            tma_load(&mQ, &bar_q2, sbase + P2_OFF_Q + x * TILE_BYTES + HALF_BYTES, 64, hA + x, tok_q0);
-          }
+          mbar_expect_tx(&bar_q2, 2 * GG::TB);
+          for (int x = 0; x < 2; ++x)
+            for (int hf = 0; hf < GG::NH; ++hf)
+              tma_load(&mQ, &bar_q2, sbase + P2_OFF_Q + x * GG::TB + hf * HALF_BYTES, 64 * hf, hA + x, tok_q0);
           q2 = true;
         }
         const int st = v % P2_NKS;
         if (v >= P2_NKS && !(ok = wait_b(&bar_ke[st], ((v / P2_NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
           break;
         const CUtensorMap *m = vv.grp ? &mKg : &mK;
-        const uint32_t dst = sbase + P2_OFF_K + st * TILE_BYTES;
-        mbar_expect_tx(&bar_kf[st], TILE_BYTES);
-        tma_load(m, &bar_kf[st], dst, 0, kvh, ak + kt * BN);
-        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
+        const uint32_t dst = sbase + GG::OFF_K + st * GG::TB;
+        mbar_expect_tx(&bar_kf[st], GG::TB);
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
         ++v;
       }
       for (int u = max(0, v - P2_NKS); u < v; ++u)
@@ -785,10 +799,10 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         const int st = v % P2_NVS;
         if (v >= P2_NVS && !(ok = wait_b(&bar_ve[st], ((v / P2_NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
           break;
-        const uint32_t dst = sbase + P2_OFF_V + st * TILE_BYTES;
-        mbar_expect_tx(&bar_vf[st], TILE_BYTES);
-        tma_load(&mV, &bar_vf[st], dst, 0, kvh, ak + kt * BN);
-        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
+        const uint32_t dst = sbase + GG::OFF_V + st * GG::TB;
+        mbar_expect_tx(&bar_vf[st], GG::TB);
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
         ++v;
       }
       for (int u = max(0, v - P2_NVS); u < v; ++u)
@@ -816,11 +830,11 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         }
         if (!wait_b(&bar_kf[v % P2_NKS], (v / P2_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t qaddr = sbase + P2_OFF_Q + x * TILE_BYTES;
-        const uint32_t kaddr = sbase + P2_OFF_K + (v % P2_NKS) * TILE_BYTES;
+        const uint32_t qaddr = sbase + P2_OFF_Q + x * GG::TB;
+        const uint32_t kaddr = sbase + GG::OFF_K + (v % P2_NKS) * GG::TB;
         const uint32_t scol = tmem + (uint32_t)(x * 128);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = 0; kk < GG::KSTEPS; ++kk) {
           const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
           umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
         }
@@ -834,18 +848,18 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         if (!wait_b(&bar_ph[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         if (!wait_b(&bar_vf[v % P2_NVS], (v / P2_NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t vaddr = sbase + P2_OFF_V + (v % P2_NVS) * TILE_BYTES;
+        const uint32_t vaddr = sbase + GG::OFF_V + (v % P2_NVS) * GG::TB;
         const uint32_t pcol = tmem + (uint32_t)(x * 128);
-        const uint32_t ocol = tmem + COL_O + (uint32_t)(x * 128);
+        const uint32_t ocol = tmem + COL_O + (uint32_t)(x * D);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV,
+          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), GG::IDESC_PV,
                   (v > 0 || kk > 0) ? 1u : 0u);
         if (!wait_b(&bar_pr[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 4; kk < 8; ++kk)
-          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV, 1u);
+          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), GG::IDESC_PV, 1u);
         umma_commit(&bar_od[x]);
         if (x == 1) umma_commit(&bar_ve[v % P2_NVS]);
         return true;
@@ -866,7 +880,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t scol = tmem + lane_base + (uint32_t)(hx * 128);
-    const uint32_t ocol = tmem + lane_base + COL_O + (uint32_t)(hx * 128);
+    const uint32_t ocol = tmem + lane_base + COL_O + (uint32_t)(hx * D);
     const int i = t.i0 + r;
     const int h = hA + hx;
     bool ok = true;
@@ -874,14 +888,18 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       // rotate this head's query tile in place: Q_g = R(f(i) - i) Q~
       ok = __all_sync(0xffffffffu, wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
       if (ok) {
-        uint8_t *qt = gbase + P2_OFF_Q + hx * TILE_BYTES;
-        for (int kk = 0; kk < 8; ++kk) {
+        uint8_t *qt = gbase + P2_OFF_Q + hx * GG::TB;
+        // pair k = (element k, element k + D/2).  D = 128: chunk u of box 0
+        // pairs with the same chunk of box 1.  D = 64: in the one 128-byte
+        // row, logical chunk lc (elements 8 lc ..) pairs with chunk lc + 4.
+        for (int kk = 0; kk < (D == 128 ? 8 : 4); ++kk) {
           const int u = r + 128 * kk;
-          const int row = u >> 3;
-          const int lc = (u & 7) ^ (row & 7);
+          const int row = D == 128 ? u >> 3 : u >> 2;
+          const int lc = D == 128 ? (u & 7) ^ (row & 7) : u & 3;
           const int n = corr_n(t.off + min(t.i0 + row, L - 1), t.G);
-          uint4 *qa = reinterpret_cast<uint4 *>(qt + u * 16);
-          uint4 *qb = reinterpret_cast<uint4 *>(qt + HALF_BYTES + u * 16);
+          uint4 *qa = reinterpret_cast<uint4 *>(D == 128 ? qt + u * 16 : qt + row * 128 + ((lc ^ (row & 7)) << 4));
+          uint4 *qb = reinterpret_cast<uint4 *>(D == 128 ? qt + HALF_BYTES + u * 16
+                                                         : qt + row * 128 + (((lc + 4) ^ (row & 7)) << 4));
           uint4 xa = *qa, xb = *qb;
           uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
 #pragma unroll
@@ -960,7 +978,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
             m_run = m_new;
           }
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t rr[32];
             tmem_ld32(ocol + c4 * 32, rr);
             tmem_wait_ld_regs(rr);
@@ -1025,9 +1043,9 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool row_ok = i < L;
-      __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * HD;
+      __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * D;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t rr[32];
         tmem_ld32(ocol + c4 * 32, rr);
         tmem_wait_ld_regs(rr);
@@ -1065,12 +1083,12 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
 // ------------------------------------------------------------------ host
 namespace {
 
-// [T, H, 128] bf16 viewed as a 3-D tensor (d, head, token); box 64 x 1 x 128.
-bool make_map(CUtensorMap *m, const void *base, int T, int H) {
+// [T, H, D] bf16 viewed as a 3-D tensor (d, head, token); box 64 x 1 x 128.
+bool make_map(CUtensorMap *m, const void *base, int T, int H, int D) {
   EncodeTiledFn enc = get_encode_tiled();
   if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)tc::HD, (cuuint64_t)H, (cuuint64_t)T};
-  cuuint64_t strides[2] = {(cuuint64_t)tc::HD * 2, (cuuint64_t)H * tc::HD * 2};
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
   cuuint32_t box[3] = {64, 1, (cuuint32_t)tc::BM};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
@@ -1096,21 +1114,26 @@ EncodeTiledFn get_encode_tiled() {
 }
 
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags) {
-  (void)batch; (void)Hq; (void)D; (void)flags;
-  return 256 + a256((size_t)T_total * Hkv * tc::HD * 2);
+  (void)batch; (void)Hq; (void)flags;
+  return 256 + a256((size_t)T_total * Hkv * D * 2);
 }
 
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
                               const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
-                              int max_seqlen, int Hq, int Hkv, long long w_pre, int w0, int window,
+                              int max_seqlen, int Hq, int Hkv, int D, long long w_pre, int w0, int window,
                               const InvFreq &inv, int plain, uint32_t flags, void *ws, size_t ws_bytes,
                               cudaStream_t st, const char **why) {
   (void)flags; (void)ws_bytes;
+  const bool pair_heads = ((Hq / Hkv) % 2) == 0;  // two heads of one GQA group per CTA
+  if (!(D == 128 || (D == 64 && pair_heads))) {
+    *why = "tensor-core prefill: head_dim 128, or 64 with an even GQA group";
+    return cudaErrorInvalidValue;
+  }
   int *err = reinterpret_cast<int *>(ws);
   __nv_bfloat16 *kg = reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(ws) + 256);
   CUtensorMap mQ, mK, mV, mKg;
-  if (!make_map(&mQ, q, T_total, Hq) || !make_map(&mK, k, Tk, Hkv) || !make_map(&mV, v, Tk, Hkv) ||
-      !make_map(&mKg, kg, Tk, Hkv)) {
+  if (!make_map(&mQ, q, T_total, Hq, D) || !make_map(&mK, k, Tk, Hkv, D) || !make_map(&mV, v, Tk, Hkv, D) ||
+      !make_map(&mKg, kg, Tk, Hkv, D)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
@@ -1118,19 +1141,20 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   if (e != cudaSuccess) return e;
   // grouped keys are needed unless the window keeps every visible pair local
   if (!plain && !(window > 0 && window <= w0)) {
-    const long long n = (long long)Tk * 8;
+    const long long n = (long long)Tk * (D / 16);
     tc::prerotate_k_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
-        (const __nv_bfloat16 *)k, kg, cu_k, batch, Tk, Hkv, w_pre, inv);
+        (const __nv_bfloat16 *)k, kg, D, cu_k, batch, Tk, Hkv, w_pre, inv);
     if ((e = cudaGetLastError()) != cudaSuccess) {
       *why = "pre-rotation launch";
       return e;
     }
   }
-  const bool pair_heads = ((Hq / Hkv) % 2) == 0;  // two heads of one GQA group per CTA
-  e = pair_heads ? cudaFuncSetAttribute(tc::bifocal_prefill2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        tc::P2_SMEM_ALLOC)
-                 : cudaFuncSetAttribute(tc::bifocal_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        tc::SMEM_ALLOC);
+  e = !pair_heads   ? cudaFuncSetAttribute(tc::bifocal_prefill_kernel,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC)
+      : D == 128 ? cudaFuncSetAttribute(tc::bifocal_prefill2_kernel<128>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Geo<128>::SMEM_ALLOC)
+                 : cudaFuncSetAttribute(tc::bifocal_prefill2_kernel<64>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Geo<64>::SMEM_ALLOC);
   if (e != cudaSuccess) {
     *why = "smem attribute";
     return e;
@@ -1150,10 +1174,15 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   p.out = (__nv_bfloat16 *)out;
   p.lse = lse;
   p.err = err;
-  p.sl2 = 1.4426950408889634f / sqrtf((float)tc::HD);
+  p.sl2 = 1.4426950408889634f / sqrtf((float)D);
   if (pair_heads) {
     dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq / 2, batch);
-    tc::bifocal_prefill2_kernel<<<grid, tc::P2_THREADS, tc::P2_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
+    if (D == 128)
+      tc::bifocal_prefill2_kernel<128><<<grid, tc::P2_THREADS, tc::Geo<128>::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p,
+                                                                                                 inv);
+    else
+      tc::bifocal_prefill2_kernel<64><<<grid, tc::P2_THREADS, tc::Geo<64>::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p,
+                                                                                               inv);
   } else {
     dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq, batch);
     tc::bifocal_prefill_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
