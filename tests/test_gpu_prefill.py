@@ -149,14 +149,16 @@ def test_planted_needles_peaked_attention():
 
 
 D64_CASES = [
-    # (seqlens, Hq, Hkv, w_pre, w0) -- even GQA groups run the tensor-core kernel
+    # (seqlens, Hq, Hkv, w_pre, w0): even GQA groups run the two-head kernel,
+    # odd ones the one-head kernel
     ((100,), 4, 2, 40, 16),
     ((129,), 2, 1, 64, 1),
     ((777,), 8, 2, 160, 200),
     ((1500,), 4, 2, 512, 0),
     ((64, 0, 513, 1, 260), 8, 4, 128, 96),
     ((1024,), 16, 8, 4096, 64),          # G = 1
-    ((600,), 4, 4, 100, 50),             # odd group: SIMT kernel
+    ((600,), 4, 4, 100, 50),             # group of 1: one-head kernel
+    ((300, 513), 3, 1, 128, 64),         # group of 3
 ]
 
 

@@ -122,7 +122,7 @@ size_t jl_bifocal_prefill_workspace_size(int32_t batch, int32_t total_tokens, in
                                          uint32_t flags) {
   if (batch < 0 || total_tokens < 0 || n_q_heads <= 0 || n_kv_heads <= 0) return 0;
   if (n_q_heads % n_kv_heads != 0) return 0;
-  const bool tc_shape = head_dim == 128 || (head_dim == 64 && (n_q_heads / n_kv_heads) % 2 == 0);
+  const bool tc_shape = head_dim == 128 || head_dim == 64;
   if (dtype != JL_BF16 || (flags & JL_FLAG_SIMT) || !tc_shape) return 0;
   return jl::tc_prefill_workspace(batch, total_tokens, n_q_heads, n_kv_heads, head_dim, flags);
 }
@@ -156,9 +156,8 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
   const jl::InvFreq inv = make_inv_freq(head_dim, rope_theta);
   const int plain = (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0;
   cudaStream_t st = (cudaStream_t)stream;
-  // tensor cores for bf16 at head_dim 128, and at 64 when the GQA group is
-  // even (the two-heads-per-CTA kernel); the SIMT kernel otherwise
-  const bool tc_shape = head_dim == 128 || (head_dim == 64 && (n_q_heads / n_kv_heads) % 2 == 0);
+  // tensor cores for bf16 at head_dim 64 and 128; the SIMT kernel otherwise
+  const bool tc_shape = head_dim == 128 || head_dim == 64;
   const bool use_simt = dtype == JL_FP32 || (flags & JL_FLAG_SIMT) || !tc_shape;
   if (use_simt) {
     cudaError_t e = jl::launch_simt_prefill(dtype == JL_BF16, head_dim, q, k, v, out, lse, cu_seqlens_q,

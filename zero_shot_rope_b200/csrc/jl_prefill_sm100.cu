@@ -41,18 +41,11 @@ namespace tc {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
-constexpr int HD = 128;  // head_dim
-constexpr int NKS = 2;   // K ring stages
-constexpr int NVS = 2;   // V ring stages
-constexpr int TILE_BYTES = BM * HD * 2;
-constexpr int HALF_BYTES = TILE_BYTES / 2;
+constexpr int NKS = 2;   // K ring stages (one head per CTA)
+constexpr int NVS = 2;   // V ring stages (one head per CTA)
+constexpr int HALF_BYTES = BM * 64 * 2;  // one 64-column SWIZZLE_128B box of a 128-row tile
 constexpr int NUM_THREADS = 224;
 constexpr int OFF_Q = 0;
-constexpr int OFF_QG = TILE_BYTES;
-constexpr int OFF_K = 2 * TILE_BYTES;
-constexpr int OFF_V = OFF_K + NKS * TILE_BYTES;
-constexpr int SMEM_TILES = OFF_V + NVS * TILE_BYTES;
-constexpr int SMEM_ALLOC = SMEM_TILES + 1024;  // slack to align the base to 1024 B
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_O = 256;
 constexpr int HI_INF = 1 << 30;
@@ -164,6 +157,33 @@ __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) 
 constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 16);  // B (= V) is MN-major
 
+constexpr int P2_THREADS = 320;
+constexpr int P2_NKS = 3;
+constexpr int P2_NVS = 2;
+constexpr int P2_OFF_Q = 0;  // Q_A, Q_B
+
+// Tile geometry for a head_dim D (64 or 128): a tile row of D bf16 is D / 64
+// SWIZZLE_128B boxes of 64 columns (HALF_BYTES each for 128 rows).  O_x sits
+// at TMEM columns COL_O + x * D.
+template <int D>
+struct Geo {
+  static constexpr int NH = D / 64;          // 64-column boxes per tile row
+  static constexpr int TB = BM * D * 2;      // one Q, K or V tile
+  static constexpr int KSTEPS = D / 16;      // k-steps of a QK product
+  // two heads per CTA: Q_A, Q_B, the K ring, the V ring
+  static constexpr int OFF_K = P2_OFF_Q + 2 * TB;
+  static constexpr int OFF_V = OFF_K + P2_NKS * TB;
+  static constexpr int SMEM_ALLOC = OFF_V + P2_NVS * TB + 1024;
+  // one head per CTA: Q, Q_g, the K ring, the V ring
+  static constexpr int P1_OFF_QG = TB;
+  static constexpr int P1_OFF_K = 2 * TB;
+  static constexpr int P1_OFF_V = P1_OFF_K + NKS * TB;
+  static constexpr int P1_SMEM_ALLOC = P1_OFF_V + NVS * TB + 1024;
+  // kind::f16, D fp32, A/B bf16, M = 128, N = D, B (= V) MN-major
+  static constexpr uint32_t IDESC_PV =
+      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((128u >> 4) << 24);
+};
+
 // --------------------------------------------------------- tile schedule
 // A query tile: rows i0..i1 of a sequence with L queries at positions
 // off + i (off = Lk - L) over keys 0..Lk-1; G follows Lk.  W > 0 hides keys
@@ -241,6 +261,7 @@ __device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int
 }
 
 // ----------------------------------------------------------------- kernel
+template <int D>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                        const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
@@ -254,6 +275,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work item (uniform across the CTA; invalid items exit before any barrier)
+  using GG = Geo<D>;
   const int s = blockIdx.z, h = blockIdx.y;
   const int a = p.cu[s];                // first query token
   const int L = p.cu[s + 1] - a;        // queries
@@ -310,9 +332,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   if (warp == 4) {
     // ================= producer: Q, then K tiles in visit order =================
     if (lane == 0) {
-      mbar_expect_tx(&bar_q, TILE_BYTES);
-      tma_load(&mQ, &bar_q, sbase + OFF_Q, 0, h, tok_q0);
-      tma_load(&mQ, &bar_q, sbase + OFF_Q + HALF_BYTES, 64, h, tok_q0);
+      mbar_expect_tx(&bar_q, GG::TB);
+      for (int hf = 0; hf < GG::NH; ++hf) tma_load(&mQ, &bar_q, sbase + OFF_Q + hf * HALF_BYTES, 64 * hf, h, tok_q0);
       int v = 0;
       bool ok = true;
       for (; v < pl.n_all; ++v) {
@@ -323,10 +344,10 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         if (v >= NKS && !(ok = wait_b(&bar_ke[st], ((v / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
           break;
         const CUtensorMap *m = vx.grp ? &mKg : &mK;
-        const uint32_t dst = sbase + OFF_K + st * TILE_BYTES;
-        mbar_expect_tx(&bar_kf[st], TILE_BYTES);
-        tma_load(m, &bar_kf[st], dst, 0, kvh, ak + kt * BN);
-        tma_load(m, &bar_kf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
+        const uint32_t dst = sbase + GG::P1_OFF_K + st * GG::TB;
+        mbar_expect_tx(&bar_kf[st], GG::TB);
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
       }
       // drain: every load issued must land before the CTA may exit
       for (int u = max(0, v - NKS); u < v; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
@@ -344,10 +365,10 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         const int st = v % NVS;
         if (v >= NVS && !(ok = wait_b(&bar_ve[st], ((v / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
           break;
-        const uint32_t dst = sbase + OFF_V + st * TILE_BYTES;
-        mbar_expect_tx(&bar_vf[st], TILE_BYTES);
-        tma_load(&mV, &bar_vf[st], dst, 0, kvh, ak + kt * BN);
-        tma_load(&mV, &bar_vf[st], dst + HALF_BYTES, 64, kvh, ak + kt * BN);
+        const uint32_t dst = sbase + GG::P1_OFF_V + st * GG::TB;
+        mbar_expect_tx(&bar_vf[st], GG::TB);
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
       }
       for (int u = max(0, v - NVS); u < v; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
     }
@@ -362,11 +383,11 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         if (!wait_b(&bar_vf[vs_], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         if (!wait_b(&bar_pr[u & 1], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t vaddr = sbase + OFF_V + vs_ * TILE_BYTES;
+        const uint32_t vaddr = sbase + GG::P1_OFF_V + vs_ * GG::TB;
         const uint32_t pcol = tmem + (uint32_t)((u & 1) * 128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + COL_O, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), IDESC_PV,
+          umma_ts(tmem + COL_O, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), GG::IDESC_PV,
                   (u > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bar_ve[vs_]);
         umma_commit(&bar_od);
@@ -384,11 +405,11 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
           const int st = v % NKS;
           if (!(ok = wait_b(&bar_kf[st], (v / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
           tc_fence_after();
-          const uint32_t qaddr = sbase + (vx.grp ? OFF_QG : OFF_Q);
-          const uint32_t kaddr = sbase + OFF_K + st * TILE_BYTES;
+          const uint32_t qaddr = sbase + (vx.grp ? GG::P1_OFF_QG : OFF_Q);
+          const uint32_t kaddr = sbase + GG::P1_OFF_K + st * GG::TB;
           const uint32_t scol = tmem + (uint32_t)((v & 1) * 128);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < GG::KSTEPS; ++kk) {
             const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
             umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
           }
@@ -412,13 +433,18 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       // rotate the query tile into grouped positions: Q_g = R(f(i) - i) Q~
       ok = __all_sync(0xffffffffu, wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
       if (ok) {
-        for (int kk = 0; kk < 8; ++kk) {
-          const int u = r + 128 * kk;        // 16-byte chunk of the first half
-          const int row = u >> 3;
-          const int lc = (u & 7) ^ (row & 7);  // logical 8-column group
+        // pair k = (element k, element k + D/2): D = 128, chunk u of box 0
+        // and the same chunk of box 1; D = 64, logical chunk lc and lc + 4 of
+        // the one 128-byte row
+        for (int kk = 0; kk < (D == 128 ? 8 : 4); ++kk) {
+          const int u = r + 128 * kk;
+          const int row = D == 128 ? u >> 3 : u >> 2;
+          const int lc = D == 128 ? (u & 7) ^ (row & 7) : u & 3;  // logical 8-column group
           const int n = corr_n(t.off + min(t.i0 + row, L - 1), t.G);
-          uint4 xa = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + u * 16);
-          uint4 xb = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + HALF_BYTES + u * 16);
+          const int oa = D == 128 ? u * 16 : row * 128 + ((lc ^ (row & 7)) << 4);
+          const int ob = D == 128 ? HALF_BYTES + u * 16 : row * 128 + (((lc + 4) ^ (row & 7)) << 4);
+          uint4 xa = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + oa);
+          uint4 xb = *reinterpret_cast<const uint4 *>(gbase + OFF_Q + ob);
           uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
@@ -434,8 +460,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
             pa[e2] = *reinterpret_cast<uint32_t *>(&ra);
             pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
           }
-          *reinterpret_cast<uint4 *>(gbase + OFF_QG + u * 16) = xa;
-          *reinterpret_cast<uint4 *>(gbase + OFF_QG + HALF_BYTES + u * 16) = xb;
+          *reinterpret_cast<uint4 *>(gbase + GG::P1_OFF_QG + oa) = xa;
+          *reinterpret_cast<uint4 *>(gbase + GG::P1_OFF_QG + ob) = xb;
         }
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -499,7 +525,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
             m_run = m_new;
           }
 #pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
+          for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t rr[32];
             tmem_ld32(tmem + lane_base + COL_O + c4 * 32, rr);
             tmem_wait_ld_regs(rr);
@@ -542,9 +568,9 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool row_ok = i < L;
-      __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * HD;
+      __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * D;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t rr[32];
         tmem_ld32(tmem + lane_base + COL_O + c4 * 32, rr);
         tmem_wait_ld_regs(rr);
@@ -656,27 +682,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // visit.  The query tiles are rotated in place into grouped positions for
 // the first phase and re-loaded by TMA for the second.
 // ===========================================================================
-constexpr int P2_THREADS = 320;
-constexpr int P2_NKS = 3;
-constexpr int P2_NVS = 2;
-constexpr int P2_OFF_Q = 0;  // Q_A, Q_B
-
-// Tile geometry for a head_dim D (64 or 128): a tile row of D bf16 is D / 64
-// SWIZZLE_128B boxes of 64 columns (HALF_BYTES each for 128 rows).  O_x sits
-// at TMEM columns COL_O + x * D.
-template <int D>
-struct Geo {
-  static constexpr int NH = D / 64;          // 64-column boxes per tile row
-  static constexpr int TB = BM * D * 2;      // one Q, K or V tile
-  static constexpr int KSTEPS = D / 16;      // k-steps of a QK product
-  static constexpr int OFF_K = P2_OFF_Q + 2 * TB;
-  static constexpr int OFF_V = OFF_K + P2_NKS * TB;
-  static constexpr int SMEM_ALLOC = OFF_V + P2_NVS * TB + 1024;
-  // kind::f16, D fp32, A/B bf16, M = 128, N = D, B (= V) MN-major
-  static constexpr uint32_t IDESC_PV =
-      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((128u >> 4) << 24);
-};
-
 template <int D>
 __global__ void __launch_bounds__(P2_THREADS, 1)
 bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
@@ -1125,8 +1130,8 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
                               cudaStream_t st, const char **why) {
   (void)flags; (void)ws_bytes;
   const bool pair_heads = ((Hq / Hkv) % 2) == 0;  // two heads of one GQA group per CTA
-  if (!(D == 128 || (D == 64 && pair_heads))) {
-    *why = "tensor-core prefill: head_dim 128, or 64 with an even GQA group";
+  if (D != 128 && D != 64) {
+    *why = "tensor-core prefill: head_dim 64 or 128";
     return cudaErrorInvalidValue;
   }
   int *err = reinterpret_cast<int *>(ws);
@@ -1149,8 +1154,12 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
       return e;
     }
   }
-  e = !pair_heads   ? cudaFuncSetAttribute(tc::bifocal_prefill_kernel,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_ALLOC)
+  e = !pair_heads   ? (D == 128 ? cudaFuncSetAttribute(tc::bifocal_prefill_kernel<128>,
+                                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                          tc::Geo<128>::P1_SMEM_ALLOC)
+                                  : cudaFuncSetAttribute(tc::bifocal_prefill_kernel<64>,
+                                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                          tc::Geo<64>::P1_SMEM_ALLOC))
       : D == 128 ? cudaFuncSetAttribute(tc::bifocal_prefill2_kernel<128>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, tc::Geo<128>::SMEM_ALLOC)
                  : cudaFuncSetAttribute(tc::bifocal_prefill2_kernel<64>,
@@ -1185,7 +1194,12 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
                                                                                                inv);
   } else {
     dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq, batch);
-    tc::bifocal_prefill_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p, inv);
+    if (D == 128)
+      tc::bifocal_prefill_kernel<128><<<grid, tc::NUM_THREADS, tc::Geo<128>::P1_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg,
+                                                                                                  p, inv);
+    else
+      tc::bifocal_prefill_kernel<64><<<grid, tc::NUM_THREADS, tc::Geo<64>::P1_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p,
+                                                                                                inv);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) *why = "tensor-core prefill launch";
