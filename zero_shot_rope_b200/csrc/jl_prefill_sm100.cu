@@ -11,16 +11,20 @@
 // each, complementary masks) on the tile that straddles d = w0; one online
 // softmax runs over all visits.
 //
-// Per CTA: one 128-row query tile of one query head, head_dim 128.
+// Two kernels, both templated on the head_dim D (64 or 128):
+// bifocal_prefill2_kernel takes two query heads of one GQA group per CTA
+// (even groups; its layout is described above its definition), and
+// bifocal_prefill_kernel one head per CTA:
 //   warps 0-3  softmax / correction / epilogue: thread r owns query row r and
 //              TMEM lane r; also rotates the query tile into grouped
 //              positions once (R(f(i) - i), §2 "Rotação de Correção").
-//   warp 4     TMA producer of Q and K tiles (128 x 128 bf16, SWIZZLE_128B).
+//   warp 4     TMA producer of Q and K tiles (128 rows x D bf16, SWIZZLE_128B
+//              boxes of 64 columns).
 //   warp 5     TMEM allocator and the single-thread tcgen05.mma issuer:
 //              S = Q K^T (SS form) into a double-buffered TMEM S, then
 //              O += P V with P read from TMEM (TS form).
 //   warp 6     TMA producer of V tiles.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384) (fp32, lane = row);
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D) (fp32, lane = row);
 // P (bf16 pairs) overwrites the first 64 columns of its S buffer.
 //
 // The grouped keys K_g = R(f(j) - j) K~ are produced once per key by
@@ -677,7 +681,7 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 //   warps 0-3 / 4-7  softmax of head A / head B (thread = row = TMEM lane)
 //   warp 8           TMA producers: lane 0 streams Q and K tiles, lane 1 V tiles
 //   warp 9           TMEM allocator and tcgen05.mma issuer
-// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 // Visit order: every grouped visit (ascending key tile), then every base
 // visit.  The query tiles are rotated in place into grouped positions for
 // the first phase and re-loaded by TMA for the second.
