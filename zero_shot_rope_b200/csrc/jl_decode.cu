@@ -456,12 +456,12 @@ static cudaError_t launch_decode_d(int GS, const CUtensorMap &mK, const CUtensor
 }
 
 void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk);
-cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
+cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
                              const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
                              int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
                              float *part_ml, int *err, cudaStream_t st);
 
-static bool use_tc_decode(bool bf16, int D, int GS) { return bf16 && D == 128 && GS <= 8; }
+static bool use_tc_decode(bool bf16, int D, int GS) { return bf16 && (D == 128 || D == 64) && GS <= 8; }
 
 // Rows of split partials the workspace must hold: a bound on the split count
 // of every plan either decode kernel may use for any key count up to
@@ -477,12 +477,12 @@ size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
   return (size_t)batch * Hq * ns;
 }
 
-static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv) {
+static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv, int D) {
   // bf16 cache viewed as (d, head, row); 64 x 1 x 128 boxes, 128-byte swizzle
   EncodeTiledFn enc = get_encode_tiled();
   if (enc == nullptr) return false;
-  cuuint64_t dims[3] = {128, (cuuint64_t)Hkv, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {256, (cuuint64_t)Hkv * 256};
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
   cuuint32_t box[3] = {64, 1, 128};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
@@ -499,14 +499,18 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
   const int keys = window > 0 ? min(max_seqlen, window) : max_seqlen;
   if (use_tc_decode(bf16, D, GS)) {
     CUtensorMap tK, tV;
-    if (!make_tile_map(&tK, kc, B * Lcap, Hkv) || !make_tile_map(&tV, vc, B * Lcap, Hkv))
+    if (!make_tile_map(&tK, kc, B * Lcap, Hkv, D) || !make_tile_map(&tV, vc, B * Lcap, Hkv, D))
       return cudaErrorInvalidValue;
     int ns, chunk;
     decode_tc_plan(B, Hkv, keys, &ns, &chunk);
-    cudaError_t e = launch_decode_tc(GS, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, Hq, Hkv, w_pre, w0,
+    cudaError_t e = launch_decode_tc(GS, D, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, Hq, Hkv, w_pre, w0,
                                      window, inv, plain, ns, chunk, part_o, part_ml, err, st);
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<__nv_bfloat16, 128><<<B * Hq, 128, 0, st>>>(part_o, part_ml, ns, (__nv_bfloat16 *)out,
+    if (D == 128)
+      decode_combine_kernel<__nv_bfloat16, 128><<<B * Hq, 128, 0, st>>>(part_o, part_ml, ns,
+                                                                        (__nv_bfloat16 *)out, lse);
+    else
+      decode_combine_kernel<__nv_bfloat16, 64><<<B * Hq, 64, 0, st>>>(part_o, part_ml, ns, (__nv_bfloat16 *)out,
                                                                       lse);
     return cudaGetLastError();
   }

@@ -37,24 +37,39 @@ namespace jl {
 namespace dtc {
 
 constexpr int TK = 128;   // keys per tile
-constexpr int HD = 128;   // head_dim
 constexpr int NROT = 8;                          // rotation warps
 constexpr int THREADS = 128 + NROT * 32 + 64;   // softmax + rotation + TMA + MMA
 constexpr int WARP_TMA = 4 + NROT;
 constexpr int WARP_MMA = 5 + NROT;
-constexpr int ROT_ROWS = TK * 8 / (NROT * 32);  // rows per rotation thread per tile
 
 constexpr int NKS = 3;    // K ring stages
 constexpr int NVS = 3;    // V ring stages
-constexpr int TILE_BYTES = TK * HD * 2;
-constexpr int HALF_BYTES = TILE_BYTES / 2;
-constexpr int OPB = 16 * 128 * 2;  // a 16-row operand (Q or P): 2 halves x 16 rows x 128 B
-constexpr int OFF_K = 0;
-constexpr int OFF_V = NKS * TILE_BYTES;
-constexpr int OFF_Q = OFF_V + NVS * TILE_BYTES;
-constexpr int OFF_P = OFF_Q + OPB;
-constexpr int SMEM_USED = OFF_P + 2 * OPB;
-constexpr int SMEM_ALLOC = SMEM_USED + 1024;
+constexpr int HALF_BYTES = TK * 64 * 2;  // one 64-column SWIZZLE_128B box of a 128-row tile
+constexpr int POPB = 16 * 128 * 2;       // the P operand: 16 rows x 128 keys (2 boxes)
+
+// Geometry for a head_dim D (64 or 128).  A K or V tile row is D / 64 boxes;
+// the Q operand is 16 rows x D.  PV is O^T = V^T P with M = 128: at D = 64 the
+// second 64 rows of V^T come from a 2 KB block of zeros (one 16-key k-step),
+// so O^T rows 64-127 stay zero and the TMEM layout is that of D = 128.
+template <int D>
+struct Geo {
+  static constexpr int NH = D / 64;
+  static constexpr int TB = TK * D * 2;
+  static constexpr int QOPB = 16 * D * 2;
+  static constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = NKS * TB;
+  static constexpr int OFF_Q = OFF_V + NVS * TB;
+  static constexpr int OFF_P = OFF_Q + (QOPB < 1024 ? 1024 : QOPB);
+  static constexpr int OFF_Z = OFF_P + 2 * POPB;   // zero block (D = 64)
+  static constexpr int SMEM_ALLOC = OFF_Z + (D == 64 ? 2048 : 0) + 1024;
+  // rotation warps: CPR 16-byte chunks (8 pairs) per row of the first half,
+  // RL row lanes, each thread ROT_ROWS rows of a tile at stride RL
+  static constexpr int CPR = D / 16;
+  static constexpr int RL = NROT * 32 / CPR;
+  static constexpr int ROT_ROWS = TK / RL;
+  static constexpr int NENT = 2 * (ROT_ROWS - 1) + 2;  // offset-table entries
+};
 constexpr uint32_t TMEM_COLS = 64;  // S^T 0: [0,16), S^T 1: [16,32), O^T: [32,48)
 constexpr uint32_t COL_O = 32;
 constexpr int ERR_TIMEOUT = 16;
@@ -149,7 +164,7 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float2 f) {
 // half (rows 128 B apart, chunk XOR-swizzled by row % 8)
 __device__ __forceinline__ int op_off(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-template <int GS>
+template <int GS, int D>
 __global__ void __launch_bounds__(THREADS, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                  const __grid_constant__ Args p, const __grid_constant__ InvFreq inv) {
@@ -162,8 +177,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   // [entry][cos, sin][16-byte slot]: the 8 values of a chunk sit in slots
   // 2 lc and 2 lc + 1, swapped for lc >= 4, so the 8 lanes of a phase (8
   // distinct chunks) read 8 distinct bank groups
-  __shared__ float4 otab[8][2][16];
+  __shared__ float4 otab[Geo<D>::NENT][2][16];
 
+  using GG = Geo<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   int L = p.seqlens[b];
@@ -176,8 +192,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   const int n = max(0, ke - kb);
   const size_t pidx = ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;  // + g * nsplit
   if (n == 0) {
-    for (int idx = threadIdx.x; idx < GS * HD; idx += THREADS)
-      p.part_o[(pidx + (size_t)(idx / HD) * p.nsplit) * HD + idx % HD] = 0.f;
+    for (int idx = threadIdx.x; idx < GS * D; idx += THREADS)
+      p.part_o[(pidx + (size_t)(idx / D) * p.nsplit) * D + idx % D] = 0.f;
     if (threadIdx.x < GS) {
       p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 0] = -INFINITY;
       p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 1] = 0.f;
@@ -232,14 +248,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       for (int u = 0; u < ntiles && ok; ++u) {
         const int sk = u % NKS, sv = u % NVS;
         if (u >= NKS && !(ok = wait_b(&bar_ke[sk], ((u / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT))) break;
-        mbar_expect_tx(&bar_kf[sk], TILE_BYTES);
-        tma_load(&mK, &bar_kf[sk], sbase + OFF_K + sk * TILE_BYTES, 0, kvh, row0 + u * TK);
-        tma_load(&mK, &bar_kf[sk], sbase + OFF_K + sk * TILE_BYTES + HALF_BYTES, 64, kvh, row0 + u * TK);
+        mbar_expect_tx(&bar_kf[sk], GG::TB);
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(&mK, &bar_kf[sk], sbase + GG::OFF_K + sk * GG::TB + hf * HALF_BYTES, 64 * hf, kvh, row0 + u * TK);
         ++nk;
         if (u >= NVS && !(ok = wait_b(&bar_ve[sv], ((u / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT))) break;
-        mbar_expect_tx(&bar_vf[sv], TILE_BYTES);
-        tma_load(&mV, &bar_vf[sv], sbase + OFF_V + sv * TILE_BYTES, 0, kvh, row0 + u * TK);
-        tma_load(&mV, &bar_vf[sv], sbase + OFF_V + sv * TILE_BYTES + HALF_BYTES, 64, kvh, row0 + u * TK);
+        mbar_expect_tx(&bar_vf[sv], GG::TB);
+        for (int hf = 0; hf < GG::NH; ++hf)
+          tma_load(&mV, &bar_vf[sv], sbase + GG::OFF_V + sv * GG::TB + hf * HALF_BYTES, 64 * hf, kvh, row0 + u * TK);
         ++nv;
       }
       for (int u = max(0, nk - NKS); u < nk; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT);
@@ -260,12 +276,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         if (uq < ntiles && uq - up < 2 && mbar_test(&bar_kr[uq % NKS], (uq / NKS) & 1)) {
           fence_after();
           const int sk = uq % NKS;
-          const uint32_t ka = sbase + OFF_K + sk * TILE_BYTES;
-          const uint32_t qa = sbase + OFF_Q;
+          const uint32_t ka = sbase + GG::OFF_K + sk * GG::TB;
+          const uint32_t qa = sbase + GG::OFF_Q;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < GG::KSTEPS; ++kk) {
             const uint32_t ko = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            const uint32_t qo = (kk >> 2) * (OPB / 2) + (kk & 3) * 32;
+            const uint32_t qo = (kk >> 2) * (GG::QOPB / 2) + (kk & 3) * 32;
             mma_ss(tmem + (uint32_t)((uq & 1) * 16), desc_k(ka + ko), desc_k(qa + qo), IDESC_QK, kk > 0 ? 1u : 0u);
           }
           commit(&bar_sf[uq & 1]);
@@ -277,12 +293,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
             mbar_test(&bar_vf[up % NVS], (up / NVS) & 1)) {
           fence_after();
           const int sv = up % NVS;
-          const uint32_t va = sbase + OFF_V + sv * TILE_BYTES;
-          const uint32_t pa = sbase + OFF_P + (up & 1) * OPB;
+          const uint32_t va = sbase + GG::OFF_V + sv * GG::TB;
+          const uint32_t pa = sbase + GG::OFF_P + (up & 1) * POPB;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tmem + COL_O, desc_mn(va + kk * 2048, HALF_BYTES),
-                   desc_k(pa + (kk >> 2) * (OPB / 2) + (kk & 3) * 32), IDESC_PV, (up > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            // the second 64 rows of V^T: the tile's second box, or (D = 64)
+            // the zero block, which lies after every V stage
+            const uint32_t vk = va + kk * 2048;
+            const uint32_t lbo = D == 128 ? (uint32_t)HALF_BYTES : sbase + (uint32_t)GG::OFF_Z - vk;
+            mma_ss(tmem + COL_O, desc_mn(vk, lbo), desc_k(pa + (kk >> 2) * (POPB / 2) + (kk & 3) * 32), IDESC_PV,
+                   (up > 0 || kk > 0) ? 1u : 0u);
+          }
           commit(&bar_ve[sv]);
           commit(&bar_od);
           ++up;
@@ -305,28 +326,45 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     }
   } else if (warp >= 4) {
     // ======================= rotation warps =======================
-    // Thread t owns one 16-byte column chunk (8 pairs) of rows r0 + RS m of
-    // every tile.  Its row-r0 rotation (the tile base) advances once per tile;
-    // the other rows compose the base with a fixed offset rotation, so the
-    // rows of a tile do not wait on one another.  With J = j0 + r0 and
-    // rho = J mod G, the offset of row m is
-    //   n(J + RS m) - n(J) = RS m - floor(RS m / G) - [rho + (RS m mod G) >= G]
+    // Thread t owns one 16-byte chunk (8 pairs) of the first half of rows
+    // r0 + RL m of every tile, together with the partner chunk of the second
+    // half (elements k + D/2).  Its row-r0 rotation (the tile base) advances
+    // once per tile; the other rows compose the base with a fixed offset
+    // rotation, so the rows of a tile do not wait on one another.  With
+    // J = j0 + r0 and rho = J mod G, the offset of row m is
+    //   n(J + RL m) - n(J) = RL m - floor(RL m / G) - [rho + (RL m mod G) >= G]
     // and the base advances by TK - floor(TK / G) - [rho + (TK mod G) >= G]:
     // each a choice between two increments, tabulated once per CTA.
-    static_assert(ROT_ROWS == 4, "offset table holds rows 1..3");
-    constexpr int RS = TK / ROT_ROWS;  // row stride of one thread (32)
+    constexpr int RS = GG::RL;        // row stride of one thread
+    constexpr int NR = GG::ROT_ROWS;  // rows of one thread per tile
+    constexpr int EB = GG::NENT - 2;  // first base-advance entry
     const int t = threadIdx.x - 128;
-    const int pc = t & 7;           // physical 16-byte chunk within a 128-byte row
-    const int r0 = t >> 3;          // first row (0..RS-1); rows r0 + RS m
-    const int lc = pc ^ (r0 & 7);   // logical chunk: pairs k = 8 lc .. 8 lc + 7
-    float bc[8], bs[8];             // rotation of row r0 of the current tile
-    int rho = 0, sm1 = 0, sm2 = 0, sm3 = 0, sb = 0;
+    int r0, lc;                       // first row; logical chunk (pairs 8 lc ..)
+    if constexpr (D == 128) {
+      r0 = t >> 3;
+      lc = (t & 7) ^ (r0 & 7);        // 8 lanes of a phase: 8 chunks of one row
+    } else {
+      // 8 lanes of a phase: rows a and a + 4 (their swizzles differ by 4, so
+      // the 4 + 4 chunks they touch fall in distinct bank groups)
+      const int ph = t >> 3;
+      r0 = ((ph >> 2) << 3) + (ph & 3) + 4 * ((t >> 2) & 1);
+      lc = t & 3;
+    }
+    // byte offsets in a tile row of this thread's two chunks (rows r0 + RS m
+    // share r0's swizzle: RS is a multiple of 8)
+    const int offa = D == 128 ? ((lc ^ (r0 & 7)) << 4) : ((lc ^ (r0 & 7)) << 4);
+    const int offb = D == 128 ? HALF_BYTES + ((lc ^ (r0 & 7)) << 4) : (((lc + 4) ^ (r0 & 7)) << 4);
+    float bc[8], bs[8];               // rotation of row r0 of the current tile
+    int rho = 0, sb = 0;
+    int smm[NR];
+#pragma unroll
+    for (int m = 0; m < NR; ++m) smm[m] = 0;
     if (bif) {
-      if (t < 64) {
-        // offset table: entries 2(m-1) + carry for rows m = 1..3, 6 + carry
+      if (t < GG::NENT * GG::CPR) {
+        // offset table: entries 2(m-1) + carry for rows m = 1..NR-1, EB + carry
         // for the base advance
-        const int tl = t & 7, en = t >> 3;
-        const int span = en < 6 ? RS * (en / 2 + 1) : TK;
+        const int tl = t % GG::CPR, en = t / GG::CPR;
+        const int span = en < EB ? RS * (en / 2 + 1) : TK;
         const int d = span - span / G - (en & 1);
         float c[8], sn[8];
 #pragma unroll
@@ -342,9 +380,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
 #pragma unroll
       for (int e = 0; e < 8; ++e) angle_cs(corr_n(jf, G) - ni, inv.v[lc * 8 + e], bc[e], bs[e]);
       rho = jf % G;
-      sm1 = RS % G;
-      sm2 = (2 * RS) % G;
-      sm3 = (3 * RS) % G;
+#pragma unroll
+      for (int m = 1; m < NR; ++m) smm[m] = (RS * m) % G;
       sb = TK % G;
       asm volatile("bar.sync 2, %0;" ::"n"(NROT * 32) : "memory");
     }
@@ -372,7 +409,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     auto advance_base = [&]() {
       const int cy = rho + sb >= G ? 1 : 0;
       float c[8], sn[8];
-      compose(6 + cy, c, sn);
+      compose(EB + cy, c, sn);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         bc[e] = c[e];
@@ -387,9 +424,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       if (!ok) break;
       const int j0 = kb + u * TK;
       if (bif && j0 < j_local) {
-        uint8_t *kt = gbase + OFF_K + sk * TILE_BYTES;
+        uint8_t *kt = gbase + GG::OFF_K + sk * GG::TB;
 #pragma unroll
-        for (int m = 0; m < ROT_ROWS; ++m) {
+        for (int m = 0; m < NR; ++m) {
           const int r = r0 + RS * m;
           if (j0 + r < j_local) {
             float rc[8], rs[8];
@@ -400,11 +437,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
                 rs[e] = bs[e];
               }
             } else {
-              const int smm = m == 1 ? sm1 : (m == 2 ? sm2 : sm3);
-              compose(2 * (m - 1) + (rho + smm >= G ? 1 : 0), rc, rs);
+              compose(2 * (m - 1) + (rho + smm[m] >= G ? 1 : 0), rc, rs);
             }
-            uint4 *pa = reinterpret_cast<uint4 *>(kt + r * 128 + pc * 16);
-            uint4 *pb = reinterpret_cast<uint4 *>(kt + HALF_BYTES + r * 128 + pc * 16);
+            uint4 *pa = reinterpret_cast<uint4 *>(kt + r * 128 + offa);
+            uint4 *pb = reinterpret_cast<uint4 *>(kt + r * 128 + offb);
             uint4 xa = *pa, xb = *pb;
             uint32_t *ua = reinterpret_cast<uint32_t *>(&xa), *ub = reinterpret_cast<uint32_t *>(&xb);
 #pragma unroll
@@ -431,24 +467,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     // ======================= softmax warpgroup =======================
     const int r = threadIdx.x;  // key row of the tile / head-dim row of O^T / TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float sl2 = rsqrtf((float)HD) * 1.4426950408889634f;
+    const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
     // Q operand: rows h < GS hold the query heads, rows GS..15 zero; also zero
-    // the padding rows of both P buffers
+    // the padding rows of both P buffers, and (D = 64) the zero block
     {
       const int h = r >> 3, c = r & 7;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
+      for (int hf = 0; hf < GG::NH; ++hf) {
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
         if (h < GS)
-          val = *reinterpret_cast<const uint4 *>(p.q + ((size_t)b * p.Hq + (size_t)kvh * GS + h) * HD + hf * 64 +
+          val = *reinterpret_cast<const uint4 *>(p.q + ((size_t)b * p.Hq + (size_t)kvh * GS + h) * D + hf * 64 +
                                                  c * 8);
-        *reinterpret_cast<uint4 *>(gbase + OFF_Q + hf * (OPB / 2) + op_off(h, c)) = val;
-        if (h >= GS)
+        *reinterpret_cast<uint4 *>(gbase + GG::OFF_Q + hf * (GG::QOPB / GG::NH) + op_off(h, c)) = val;
+      }
+      if (h >= GS)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
           for (int pb = 0; pb < 2; ++pb)
-            *reinterpret_cast<uint4 *>(gbase + OFF_P + pb * OPB + hf * (OPB / 2) + op_off(h, c)) =
+            *reinterpret_cast<uint4 *>(gbase + GG::OFF_P + pb * POPB + hf * (POPB / 2) + op_off(h, c)) =
                 make_uint4(0u, 0u, 0u, 0u);
-      }
+      if constexpr (D == 64) reinterpret_cast<uint4 *>(gbase + GG::OFF_Z)[r] = make_uint4(0u, 0u, 0u, 0u);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bar_q);
     }
@@ -523,7 +562,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         for (int g = 0; g < GS; ++g) l_part[g] *= f[g];
       }
       // P (bf16) into the B operand of the PV MMA: row g = head, column r = key
-      uint8_t *pbuf = gbase + OFF_P + bsel * OPB + (r >> 6) * (OPB / 2);
+      uint8_t *pbuf = gbase + GG::OFF_P + bsel * POPB + (r >> 6) * (POPB / 2);
       const int chunk = (r & 63) >> 3;
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
@@ -537,12 +576,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         const int sv = u % NVS;
         wait_b(&bar_vf[sv], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT);
         if (!valid && !abort_flag) {
-          uint8_t *vt = gbase + OFF_V + sv * TILE_BYTES;
+          uint8_t *vt = gbase + GG::OFF_V + sv * GG::TB;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            *reinterpret_cast<uint4 *>(vt + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4 *>(vt + HALF_BYTES + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
+          for (int hf = 0; hf < GG::NH; ++hf)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4 *>(vt + hf * HALF_BYTES + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       // last tile: PV of the previous tile must be complete before this
@@ -571,15 +610,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       fence_after();
       uint32_t orow[8];
       tmem_ld8(tmem + lane_base + COL_O, orow);
+      if (r < D)  // O^T row r is head_dim element r
 #pragma unroll
-      for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * HD + r] = __uint_as_float(orow[g]);
+        for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * D + r] = __uint_as_float(orow[g]);
       if (r < GS) {
         const float l = lred[0][r] + lred[1][r] + lred[2][r] + lred[3][r];
         p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 0] = m_run[r];
         p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 1] = l;
       }
     } else {
-      for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * HD + r] = 0.f;
+      if (r < D)
+        for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * D + r] = 0.f;
       if (r < GS) {
         p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 0] = -INFINITY;
         p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 1] = 0.f;
@@ -609,7 +650,7 @@ void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk)
   *nsplit = (maxL + c - 1) / c;
 }
 
-cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
+cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
                              const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
                              int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
                              float *part_ml, int *err, cudaStream_t st) {
@@ -630,17 +671,29 @@ cudaError_t launch_decode_tc(int GS, const CUtensorMap &mK, const CUtensorMap &m
   a.err = err;
   dim3 grid(nsplit, Hkv, B);
   cudaError_t e;
-#define JL_DTC(GG)                                                                                       \
-  e = cudaFuncSetAttribute(dtc::decode_tc_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,         \
-                           dtc::SMEM_ALLOC);                                                              \
-  if (e != cudaSuccess) return e;                                                                        \
-  dtc::decode_tc_kernel<GG><<<grid, dtc::THREADS, dtc::SMEM_ALLOC, st>>>(mK, mV, a, inv);
-  switch (GS) {
-    case 1: JL_DTC(1) break;
-    case 2: JL_DTC(2) break;
-    case 4: JL_DTC(4) break;
-    case 8: JL_DTC(8) break;
-    default: return cudaErrorInvalidValue;
+#define JL_DTC(GG, DD)                                                                                    \
+  e = cudaFuncSetAttribute(dtc::decode_tc_kernel<GG, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
+                           dtc::Geo<DD>::SMEM_ALLOC);                                                        \
+  if (e != cudaSuccess) return e;                                                                          \
+  dtc::decode_tc_kernel<GG, DD><<<grid, dtc::THREADS, dtc::Geo<DD>::SMEM_ALLOC, st>>>(mK, mV, a, inv);
+  if (D == 128) {
+    switch (GS) {
+      case 1: JL_DTC(1, 128) break;
+      case 2: JL_DTC(2, 128) break;
+      case 4: JL_DTC(4, 128) break;
+      case 8: JL_DTC(8, 128) break;
+      default: return cudaErrorInvalidValue;
+    }
+  } else if (D == 64) {
+    switch (GS) {
+      case 1: JL_DTC(1, 64) break;
+      case 2: JL_DTC(2, 64) break;
+      case 4: JL_DTC(4, 64) break;
+      case 8: JL_DTC(8, 64) break;
+      default: return cudaErrorInvalidValue;
+    }
+  } else {
+    return cudaErrorInvalidValue;
   }
 #undef JL_DTC
   return cudaGetLastError();
