@@ -80,6 +80,24 @@ def test_decode_128k_steps(decode_cache, step):
     assert np.abs(po - ro).mean() > 5 * np.abs(got - ro).mean()
 
 
+@pytest.mark.parametrize("step", [0, 1])
+def test_decode_128k_head_dim_64(step):
+    """The decode workload's sizes at head_dim 64 (the tensor-core decode with
+    the zero-padded PV), steps 0 and 1 (G = 4, then 5), in full."""
+    w = synth.WORKLOADS["decode_128k"]
+    g = torch.Generator().manual_seed(640 + step)
+    cap = w.seqlens[0] + 1
+    kc = torch.randn(1, cap, w.n_kv_heads, 64, generator=g).to(torch.bfloat16)
+    vc = torch.randn(1, cap, w.n_kv_heads, 64, generator=g).to(torch.bfloat16)
+    q = torch.randn(1, w.n_q_heads, 64, generator=g).to(torch.bfloat16)
+    L = w.seqlens[0] + step
+    out, lse = decode_gpu(q, kc, vc, [L], cap, w.w_pretrained, w.w0, w.rope_theta)
+    ro, rl = oracle.bifocal_decode(q, kc, vc, [L], w.w_pretrained, w.w0, w.rope_theta)
+    assert_close(to_np(out), ro, torch.bfloat16, f"D64 step {step}")
+    assert_close(to_np(lse), rl, torch.bfloat16, f"D64 step {step} lse")
+    assert np.linalg.norm(to_np(out) - ro) / np.linalg.norm(ro) < 1e-2
+
+
 def test_decode_zero_length_writes_zero():
     dev = torch.device("cuda:0")
     q = torch.randn(2, 8, 128).to(torch.bfloat16)

@@ -188,3 +188,16 @@ def test_head_dim_64_tensor_matches_simt_and_chunks():
     ro, rl = oracle.bifocal_attention_kv(q[1300:], k, v, cu_q, cu, 512, 300, 1e4, window=900)
     assert_close(to_np(o2), ro, torch.bfloat16, "chunk out")
     assert_close(to_np(l2), rl, torch.bfloat16, "chunk lse")
+
+
+def test_full_length_head_dim_64_sampled_rows():
+    # 32K tokens, 32/8 heads, D = 64, G = 4 (the two-head kernel at head_dim 64)
+    L, Hq, Hkv, w_pre, w0 = 32768, 32, 8, 8192, 4096
+    q, k, v, cu = synth.random_case(64, (L,), Hq, Hkv, 64, torch.bfloat16)
+    out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e6)
+    rows = sample_rows([L], w0, [oracle.group_size(L, w_pre)], n_random=24, seed=64)
+    ro, rl = oracle.bifocal_attention(q, k, v, cu, w_pre, w0, 1e6, rows=rows)
+    got = to_np(out)[rows]
+    assert_close(got, ro, torch.bfloat16, "out")
+    assert_close(to_np(lse)[:, rows], rl, torch.bfloat16, "lse")
+    assert np.linalg.norm(got - ro) / np.linalg.norm(ro) < 1e-2
