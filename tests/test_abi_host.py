@@ -203,3 +203,27 @@ def test_decode_workspace_covers_every_shorter_plan(B, Hq, Hkv, D):
     sizes = [jl.jl_bifocal_decode_workspace_size(B, Hq, Hkv, D, L) for L in lens]
     assert all(x > 0 for x in sizes)
     assert all(b >= a for a, b in zip(sizes, sizes[1:]))
+
+
+def test_library_never_reaches_the_oracle():
+    # the product path (package sources and the CUDA library) neither imports
+    # nor calls the CPU oracle: there is no CPU fallback through it
+    pkg = os.path.join(ROOT, "zero_shot_rope_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dirpath, fn)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", txt, flags=re.M), fn
+                assert "bifocal_attention(" not in txt or fn.endswith((".cu", ".cuh")), fn
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the behaviour without a GPU")
+def test_calls_fail_loudly_without_a_gpu():
+    # no device: a valid call reports a CUDA error instead of computing
+    # anything on the host (there is no CPU fallback)
+    jl = _lib()
+    status = _prefill_raw(jl, ws=1 << 20, ws_bytes=1 << 30)
+    assert jl.status_string(status) == "JL_ERR_CUDA"
+    assert jl.last_error()
+    status = _decode_raw(jl)
+    assert jl.status_string(status) == "JL_ERR_CUDA"
