@@ -1,0 +1,36 @@
+/*
+ * jetlong_debug.h — a test hook of the library, not an attention entry point.
+ *
+ * jl_debug_prefill_visits — the prefill kernels' tile schedule, computed on
+ * the host by the same code the kernels run: for query tile qt (rows
+ * 128 qt .. of a sequence with L queries at positions Lk - L + i over keys
+ * 0 .. Lk-1), every (key tile, branch, mask) visit in the order the kernels
+ * process them.  The method's routing (§1 "Janela Local" / "Janela Remota"
+ * of the Jet-Long technical summary: distance d < w0 scored with the base
+ * RoPE, d >= w0 at grouped positions; a sliding window hides d >= window)
+ * must come out as: every visible (row, key) pair claimed by exactly one
+ * visit, on the right branch.
+ *   G        the group size (G = 1: no grouped visits, as in plain mode)
+ *   window   0: no window
+ *   out      host int array, 5 ints per visit: key tile, grouped (0/1),
+ *            masked (0/1), lo, hi — a masked visit keeps the columns whose
+ *            distance d satisfies lo <= d <= hi, an unmasked one all 128
+ *   cap      visits that fit in out
+ * Returns the number of visits (which may exceed cap), or -1 for arguments
+ * outside the kernels' range (L <= 0, Lk < L, w0 < 0, window < 0, G < 1, a
+ * tile past L, out NULL).  Host-only; no CUDA call.
+ */
+#ifndef JETLONG_DEBUG_H
+#define JETLONG_DEBUG_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+int jl_debug_prefill_visits(int L, int Lk, int w0, int window, int G, int qt, int *out, int cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JETLONG_DEBUG_H */

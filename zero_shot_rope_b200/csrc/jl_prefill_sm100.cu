@@ -211,7 +211,7 @@ struct VisitPlan {
   int n_grp, n_all, ks_begin, g_begin;
 };
 
-__device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
+__host__ __device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
   VisitPlan pl;
   const int pmin = t.off + t.i0, pmax = t.off + t.i1;  // row positions
   const int kt_last = pmax / BN;                        // last key tile with a visible key
@@ -244,7 +244,8 @@ __device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
   return pl;
 }
 
-__device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int w0, int v, int &kt, Visit &out) {
+__host__ __device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int w0, int v, int &kt,
+                                                  Visit &out) {
   const bool grp = v < pl.n_grp;
   kt = grp ? pl.g_begin + v : pl.ks_begin + (v - pl.n_grp);
   const int j0 = kt * BN;
@@ -1211,3 +1212,34 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
 }
 
 }  // namespace jl
+
+// Host copy of the prefill tile schedule, for tests: the visits of query tile
+// qt of a sequence with L queries over Lk keys, five ints each (key tile,
+// grouped, masked, lo, hi), at most cap visits; returns the visit count, or -1
+// for arguments outside the kernels' range.
+extern "C" int jl_debug_prefill_visits(int L, int Lk, int w0, int window, int G, int qt, int *out, int cap) {
+  using namespace jl::tc;
+  if (L <= 0 || Lk < L || w0 < 0 || window < 0 || G < 1 || qt < 0 || qt * BM >= L || out == nullptr) return -1;
+  Tile t;
+  t.L = L;
+  t.qt = qt;
+  t.i0 = qt * BM;
+  t.i1 = L - 1 < t.i0 + BM - 1 ? L - 1 : t.i0 + BM - 1;
+  t.Lk = Lk;
+  t.off = Lk - L;
+  t.W = window;
+  t.G = G;
+  t.bif = G > 1;
+  const VisitPlan pl = make_plan(t, w0);
+  for (int v = 0; v < pl.n_all && v < cap; ++v) {
+    int kt;
+    Visit vx;
+    visit_at(t, pl, w0, v, kt, vx);
+    out[5 * v + 0] = kt;
+    out[5 * v + 1] = vx.grp;
+    out[5 * v + 2] = vx.mask;
+    out[5 * v + 3] = vx.lo;
+    out[5 * v + 4] = vx.hi;
+  }
+  return pl.n_all;
+}
