@@ -29,6 +29,19 @@ extern "C" {
 
 int jl_debug_prefill_visits(int L, int Lk, int w0, int window, int G, int qt, int *out, int cap);
 
+/*
+ * jl_debug_decode_plan — the decode's split plan, computed on the host by the
+ * code the decode call uses: sequence b's keys max(0, L_b - window) .. L_b-1
+ * (all keys when window = 0) go to splits of `chunk` keys, `nsplit` per
+ * (sequence, kv head), so every length up to max_seqlen must fit in
+ * nsplit * chunk keys and the workspace's `partial_rows` must hold
+ * batch * Hq * nsplit.  bf16 != 0 selects the bf16 plan (tensor-core kernel
+ * at head_dim 64 / 128 with a GQA group <= 8), 0 the fp32 one.  Returns 0, or
+ * -1 for sizes outside the decode's range.  Host-only; no CUDA call.
+ */
+int jl_debug_decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int window, int bf16,
+                         int *nsplit, int *chunk, long long *partial_rows);
+
 #ifdef __cplusplus
 }
 #endif

@@ -620,3 +620,25 @@ extern "C" jl_status jl_bifocal_decode_noalloc(const void *q, const void *k_cach
                            head_dim, w_pretrained, w0, rope_theta, out, lse, scratch,
                            (size_t)JL_DECODE_NOALLOC_SCRATCH_BYTES, dtype, flags, stream);
 }
+
+// Host copy of the decode split plan, for tests: the plan launch_decode uses
+// for these sizes (tensor-core kernel for bf16 at head_dim 64 / 128 with a
+// GQA group <= 8, the CUDA-core kernel otherwise) and the partial rows the
+// workspace holds.  Returns 0, or -1 for sizes outside the decode's range.
+extern "C" int jl_debug_decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int window, int bf16,
+                                    int *nsplit, int *chunk, long long *partial_rows) {
+  if (batch < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128) || max_seqlen < 1 ||
+      window < 0 || nsplit == nullptr || chunk == nullptr || partial_rows == nullptr)
+    return -1;
+  const int GS = Hq / Hkv;
+  const int keys = window > 0 ? min(max_seqlen, window) : max_seqlen;
+  if (jl::use_tc_decode(bf16 != 0, D, GS)) {
+    jl::decode_tc_plan(batch, Hkv, keys, nsplit, chunk);
+  } else {
+    const jl::DecodePlan pl = jl::decode_plan(batch, Hq, Hkv, D, keys, bf16 ? 2 : 4);
+    *nsplit = pl.nsplit;
+    *chunk = pl.chunk;
+  }
+  *partial_rows = (long long)jl::decode_partial_rows(batch, Hq, Hkv, D, max_seqlen);
+  return 0;
+}
