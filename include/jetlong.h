@@ -110,6 +110,7 @@ size_t jl_bifocal_prefill_workspace_size(int32_t batch, int32_t total_tokens,
  *   cu_seqlens  [batch + 1]  device int32 prefix sums, cu[0] = 0,
  *                            cu[batch] = total_tokens, non-decreasing; a
  *                            zero-length sequence is legal and writes nothing
+ *   batch       <= 65535 sequences per call (JL_ERR_UNSUPPORTED beyond)
  *   max_seqlen  >= every sequence length (sizes the grid)
  *   head_dim    64 or 128;   n_q_heads % n_kv_heads == 0
  *   w_pretrained >= 1; w0 >= 0 (w0 = 0: every pair grouped; w0 >= L: none)
@@ -198,7 +199,7 @@ size_t jl_bifocal_decode_workspace_size(int32_t batch, int32_t n_q_heads,
  *   out        [B, Hq, D]          attention output (dtype of q)
  *   lse        [B, Hq] fp32 or NULL
  *   workspace  >= jl_bifocal_decode_workspace_size(...) bytes
- * head_dim 64 or 128; n_q_heads / n_kv_heads in {1, 2, 4, 8}.
+ * head_dim 64 or 128; n_q_heads / n_kv_heads in {1, 2, 4, 8}; batch <= 65535.
  */
 jl_status jl_bifocal_decode(const void *q, const void *k_cache,
                             const void *v_cache, const int32_t *seqlens,

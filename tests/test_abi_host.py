@@ -83,6 +83,7 @@ def _prefill_raw(jl, **kw):
     (dict(maxL=0), "JL_ERR_INVALID_ARG"),
     (dict(maxL=17), "JL_ERR_INVALID_ARG"),
     (dict(batch=-1), "JL_ERR_INVALID_ARG"),
+    (dict(batch=70000, T=70000, maxL=1), "JL_ERR_UNSUPPORTED"),
     (dict(ws=None, ws_bytes=0), "JL_ERR_WORKSPACE"),
     (dict(ws=(1 << 20) + 16, ws_bytes=1 << 30), "JL_ERR_WORKSPACE"),
 ])
@@ -124,6 +125,7 @@ def _decode_raw(jl, **kw):
     (dict(ws_bytes=16), "JL_ERR_WORKSPACE"),
     (dict(ws=(1 << 20) + 64), "JL_ERR_WORKSPACE"),
     (dict(w_pre=0), "JL_ERR_INVALID_ARG"),
+    (dict(B=70000), "JL_ERR_UNSUPPORTED"),
 ])
 def test_decode_rejects_bad_arguments_before_launch(kw, status):
     jl = _lib()

@@ -143,6 +143,8 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
   if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0)
     return fail(JL_ERR_INVALID_ARG, "batch, token counts and max_seqlen must be >= 0");
   if (batch == 0 || total_q == 0) return ok();  // nothing to attend
+  if (batch > 65535)  // the kernels' grid takes one z-block per sequence
+    return fail(JL_ERR_UNSUPPORTED, "batch %d exceeds 65535 sequences per call", batch);
   if (total_k < total_q)
     return fail(JL_ERR_INVALID_ARG, "total_k (%d) < total_q (%d): every sequence needs Lq <= Lk", total_k, total_q);
   if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr) return fail(JL_ERR_INVALID_ARG, "cu_seqlens is NULL");
@@ -216,6 +218,8 @@ jl_status jl_bifocal_decode_window(const void *q, const void *k_cache, const voi
   if (flags & ~(uint32_t)JL_FLAG_PLAIN_CAUSAL) return fail(JL_ERR_INVALID_ARG, "unknown or prefill-only flag bits 0x%x", flags);
   if (batch < 0) return fail(JL_ERR_INVALID_ARG, "batch must be >= 0");
   if (batch == 0) return ok();
+  if (batch > 65535)  // the kernels' grid takes one z-block per sequence
+    return fail(JL_ERR_UNSUPPORTED, "batch %d exceeds 65535 sequences per call", batch);
   if (cache_capacity < 1 || max_seqlen < 1 || max_seqlen > cache_capacity)
     return fail(JL_ERR_INVALID_ARG, "need 1 <= max_seqlen <= cache_capacity (got %d, %d)", max_seqlen, cache_capacity);
   if (q == nullptr || k_cache == nullptr || v_cache == nullptr || out == nullptr || seqlens == nullptr)
