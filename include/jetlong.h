@@ -246,12 +246,16 @@ jl_status jl_bifocal_decode_window(const void *q, const void *k_cache,
  * the process exits.
  *
  *   Arguments, layouts and results are those of jl_bifocal_decode, minus the
- *   workspace.  A decode whose jl_bifocal_decode_workspace_size(...) exceeds
+ *   workspace.  Arguments are checked exactly as jl_bifocal_decode checks them, first;
+ *   then a decode whose jl_bifocal_decode_workspace_size(...) exceeds
  *   JL_DECODE_NOALLOC_SCRATCH_BYTES is rejected with JL_ERR_WORKSPACE before
  *   any launch (jl_last_error() says how much it needed).
- *   The first call on a device (with that device current) looks up the
- *   array's device address once (cudaGetSymbolAddress); make that first call
- *   before any stream capture.  A failed lookup returns JL_ERR_CUDA.
+ *   The array's device address is looked up (cudaGetSymbolAddress) by the
+ *   first call made under each CUDA context and cached by that context's
+ *   unique id: a context made current through the driver API, or the primary
+ *   context re-created after cudaDeviceReset, gets its own lookup.  Make the
+ *   first call under a context before any stream capture.  A failed lookup
+ *   returns JL_ERR_CUDA.
  *   All calls share the one array, which keeps the last call's contents; the
  *   kernels clear what must start at zero.  Calls that overlap on the GPU
  *   (different streams, or different host threads, on the same device) race
@@ -268,6 +272,22 @@ jl_status jl_bifocal_decode_noalloc(const void *q, const void *k_cache,
                                     int32_t w0, double rope_theta, void *out,
                                     float *lse, jl_dtype dtype, uint32_t flags,
                                     void *stream);
+
+/*
+ * jl_bifocal_decode_noalloc_error — the kernel error word of the most recent
+ * jl_bifocal_decode_noalloc call under the current context.  (An addition of
+ * this library; the paper has no counterpart.)
+ *
+ * The decode kernels report a bounded wait that ran out (a stalled pipeline:
+ * the call returns, its output is not valid) by setting bits of a word in
+ * their scratch; with a caller workspace that is the workspace's first int32,
+ * with jl_bifocal_decode_noalloc it lives in the library's own array, which
+ * the caller cannot address.  This call enqueues one device-to-host copy of
+ * that word into *error_word (a host int32; pinned memory keeps the copy
+ * asynchronous) on `stream`; read it after synchronising the stream.  0 means
+ * no error.  NULL error_word: JL_ERR_INVALID_ARG; a failed copy: JL_ERR_CUDA.
+ */
+jl_status jl_bifocal_decode_noalloc_error(int32_t *error_word, void *stream);
 
 #ifdef __cplusplus
 } /* extern "C" */

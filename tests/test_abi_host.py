@@ -84,6 +84,7 @@ def _prefill_raw(jl, **kw):
     (dict(maxL=17), "JL_ERR_INVALID_ARG"),
     (dict(batch=-1), "JL_ERR_INVALID_ARG"),
     (dict(batch=70000, T=70000, maxL=1), "JL_ERR_UNSUPPORTED"),
+    (dict(Hq=70000, Hkv=1), "JL_ERR_UNSUPPORTED"),    # grid y extent (heads) above 65535
     (dict(ws=None, ws_bytes=0), "JL_ERR_WORKSPACE"),
     (dict(ws=(1 << 20) + 16, ws_bytes=1 << 30), "JL_ERR_WORKSPACE"),
 ])
@@ -126,6 +127,7 @@ def _decode_raw(jl, **kw):
     (dict(ws=(1 << 20) + 64), "JL_ERR_WORKSPACE"),
     (dict(w_pre=0), "JL_ERR_INVALID_ARG"),
     (dict(B=70000), "JL_ERR_UNSUPPORTED"),
+    (dict(Hq=70000, Hkv=70000), "JL_ERR_UNSUPPORTED"),  # grid y extent (kv heads) above 65535
 ])
 def test_decode_rejects_bad_arguments_before_launch(kw, status):
     jl = _lib()

@@ -67,6 +67,10 @@ jl_status check_heads(int32_t Hq, int32_t Hkv, int32_t D) {
   return JL_OK;
 }
 
+// The kernels put one head (prefill: a query head or a pair of them; decode:
+// a kv head) per y-block of their grid, whose extent is at most 65535.
+constexpr int32_t kMaxGridY = 65535;
+
 jl_status check_method(int64_t w_pre, int32_t w0, double theta) {
   if (w_pre < 1) return fail(JL_ERR_INVALID_ARG, "w_pretrained must be >= 1 (got %lld)", (long long)w_pre);
   if (w0 < 0) return fail(JL_ERR_INVALID_ARG, "w0 must be >= 0 (got %d)", w0);
@@ -135,6 +139,8 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
                                 void *workspace, size_t workspace_bytes, void *stream) {
   jl_status s;
   if ((s = check_heads(n_q_heads, n_kv_heads, head_dim)) != JL_OK) return s;
+  if (n_q_heads > kMaxGridY)
+    return fail(JL_ERR_UNSUPPORTED, "n_q_heads %d exceeds %d per call", n_q_heads, kMaxGridY);
   if ((s = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return s;
   if (window < 0) return fail(JL_ERR_INVALID_ARG, "window must be >= 0 (0: no window), got %d", window);
   if (dtype != JL_BF16 && dtype != JL_FP32) return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
@@ -210,6 +216,8 @@ jl_status jl_bifocal_decode_window(const void *q, const void *k_cache, const voi
   jl_status s;
   if (window < 0) return fail(JL_ERR_INVALID_ARG, "window must be >= 0 (0: no window), got %d", window);
   if ((s = check_heads(n_q_heads, n_kv_heads, head_dim)) != JL_OK) return s;
+  if (n_kv_heads > kMaxGridY)
+    return fail(JL_ERR_UNSUPPORTED, "n_kv_heads %d exceeds %d per call", n_kv_heads, kMaxGridY);
   const int gs = n_q_heads / n_kv_heads;
   if (gs != 1 && gs != 2 && gs != 4 && gs != 8)
     return fail(JL_ERR_UNSUPPORTED, "decode supports n_q_heads / n_kv_heads in {1,2,4,8} (got %d)", gs);

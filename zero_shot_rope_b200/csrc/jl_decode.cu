@@ -396,6 +396,13 @@ static size_t decode_smem(int elem, int D, int GS) {
   return ring > red ? ring : red;
 }
 
+// (sequence, kv head) pairs of a call, at least 1; computed in 64 bits and
+// clamped, since batch and Hkv may each be up to 65535
+static int sequence_heads(int batch, int Hkv) {
+  const long long bh = (long long)batch * (long long)Hkv;
+  return bh < 1 ? 1 : (bh > INT32_MAX ? INT32_MAX : (int)bh);
+}
+
 // Split count: one wave of CTAs (148 SMs x CTAs resident per SM), splits of at
 // least one 64-key tile, rounded to whole tiles.
 DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int elem) {
@@ -403,7 +410,7 @@ DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int el
   const int GS = Hq / Hkv;
   const int per_sm = (GS <= 4 && elem == 2) ? 2 : 1;
   const int target = 148 * per_sm;
-  const int per_bh = max(1, batch * Hkv);
+  const int per_bh = sequence_heads(batch, Hkv);
   int ns = max(1, target / per_bh);
   const int maxL = max(1, max_seqlen);
   int chunk = (maxL + ns - 1) / ns;
@@ -470,7 +477,7 @@ static bool use_tc_decode(bool bf16, int D, int GS) { return bf16 && (D == 128 |
 // per key tile.
 size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
   const int GS = Hq / Hkv;
-  const int per_bh = max(1, batch * Hkv);
+  const int per_bh = sequence_heads(batch, Hkv);
   const int tiles64 = (max(1, max_seqlen) + DEC_TK - 1) / DEC_TK;
   int ns = min(max(1, 2 * 148 / per_bh), tiles64);  // both element sizes of decode_plan
   if (use_tc_decode(true, D, GS)) ns = max(ns, min(max(1, 148 / per_bh), (max(1, max_seqlen) + 127) / 128));
@@ -567,28 +574,70 @@ void set_last_error(const char *fmt, ...);
 // File-scope scratch of JL_DECODE_NOALLOC_SCRATCH_BYTES.  Every GPU that loads
 // the library holds it until the process exits.  In host code this name is
 // only a host-side stand-in: the device address comes from
-// cudaGetSymbolAddress, taken once per device below.
+// cudaGetSymbolAddress, looked up below once per CUDA context.
 static __device__ __align__(256) uint8_t g_decode_scratch[JL_DECODE_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-std::mutex g_scratch_mu;
-void *g_scratch_addr[256] = {nullptr};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of g_decode_scratch on the current device (set up on the
-// first call made with that device current).
-cudaError_t scratch_for_current_device(void **out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+std::mutex g_scratch_mu;
+// The symbol's address belongs to the context (module instance) that was
+// current when it was looked up: a driver-API context made current by a host
+// runtime, or the primary context re-created after cudaDeviceReset, has its
+// own.  So the cache is keyed by the context's unique id, which a new context
+// never shares with an old one.
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  void *addr;
+};
+ScratchEntry g_scratch_cache[64];
+int g_scratch_n = 0;
+
+template <typename Fn>
+Fn driver_fn(const char *name) {
+  void *ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(ptr);
+}
+
+// Unique id of the context current on this thread (0 if none is current yet).
+cudaError_t current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (get_cur == nullptr || get_id == nullptr) return cudaErrorNotSupported;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  *id = 0;
+  if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+  return cudaSuccess;
+}
+
+// Device address of g_decode_scratch in the context current on this thread.
+// The first call under a context looks it up (which also makes the runtime's
+// primary context current when none was); later calls find it in the cache.
+cudaError_t scratch_for_current_context(void **out) {
+  unsigned long long id = 0;
+  cudaError_t e = current_context_id(&id);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 256) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+  for (int i = 0; i < g_scratch_n; ++i)
+    if (id != 0 && g_scratch_cache[i].ctx_id == id) {
+      *out = g_scratch_cache[i].addr;
+      return cudaSuccess;
+    }
+  void *p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess) return e;
+  if (id == 0 && (e = current_context_id(&id)) != cudaSuccess) return e;  // the lookup made one current
+  if (id != 0) {
+    // keep the newest 64 contexts; an evicted one only costs a new lookup
+    const int slot = g_scratch_n < 64 ? g_scratch_n++ : (int)(id % 64);
+    g_scratch_cache[slot] = ScratchEntry{id, p};
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return cudaSuccess;
 }
 }  // namespace
@@ -599,6 +648,13 @@ extern "C" jl_status jl_bifocal_decode_noalloc(const void *q, const void *k_cach
                                                int32_t head_dim, int64_t w_pretrained, int32_t w0,
                                                double rope_theta, void *out, float *lse, jl_dtype dtype,
                                                uint32_t flags, void *stream) {
+  // Argument checks first, exactly those of jl_bifocal_decode: a dry run with
+  // an impossible (NULL) workspace returns every argument error, and
+  // JL_ERR_WORKSPACE only once the arguments are valid.
+  jl_status s = jl_bifocal_decode(q, k_cache, v_cache, seqlens, batch, cache_capacity, max_seqlen, n_q_heads,
+                                  n_kv_heads, head_dim, w_pretrained, w0, rope_theta, out, lse, nullptr, 0, dtype,
+                                  flags, stream);
+  if (s != JL_ERR_WORKSPACE) return s;  // an argument error, or JL_OK for an empty batch
   const size_t need = jl_bifocal_decode_workspace_size(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen);
   if (need > (size_t)JL_DECODE_NOALLOC_SCRATCH_BYTES) {
     jl::set_last_error("this decode needs %zu bytes of scratch; the allocation-free entry point has a fixed %u "
@@ -606,19 +662,31 @@ extern "C" jl_status jl_bifocal_decode_noalloc(const void *q, const void *k_cach
                        need, (unsigned)JL_DECODE_NOALLOC_SCRATCH_BYTES);
     return JL_ERR_WORKSPACE;
   }
-  if (batch <= 0)  // nothing to do (or an argument error): no scratch needed
-    return jl_bifocal_decode(q, k_cache, v_cache, seqlens, batch, cache_capacity, max_seqlen, n_q_heads,
-                             n_kv_heads, head_dim, w_pretrained, w0, rope_theta, out, lse, nullptr, 0, dtype,
-                             flags, stream);
   void *scratch = nullptr;
-  const cudaError_t e = scratch_for_current_device(&scratch);
+  const cudaError_t e = scratch_for_current_context(&scratch);
   if (e != cudaSuccess) {
-    jl::set_last_error("cudaGetSymbolAddress of the decode scratch failed: %s", cudaGetErrorString(e));
+    jl::set_last_error("looking up the decode scratch address failed: %s", cudaGetErrorString(e));
     return JL_ERR_CUDA;
   }
   return jl_bifocal_decode(q, k_cache, v_cache, seqlens, batch, cache_capacity, max_seqlen, n_q_heads, n_kv_heads,
                            head_dim, w_pretrained, w0, rope_theta, out, lse, scratch,
                            (size_t)JL_DECODE_NOALLOC_SCRATCH_BYTES, dtype, flags, stream);
+}
+
+extern "C" jl_status jl_bifocal_decode_noalloc_error(int32_t *error_word, void *stream) {
+  if (error_word == nullptr) {
+    jl::set_last_error("error_word is NULL");
+    return JL_ERR_INVALID_ARG;
+  }
+  void *scratch = nullptr;
+  cudaError_t e = scratch_for_current_context(&scratch);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(error_word, scratch, sizeof(int32_t), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    jl::set_last_error("reading the decode scratch error word failed: %s", cudaGetErrorString(e));
+    return JL_ERR_CUDA;
+  }
+  return JL_OK;
 }
 
 // Host copy of the decode split plan, for tests: the plan launch_decode uses

@@ -1,5 +1,5 @@
 // Tensor-core split-KV decode kernel for Dynamic Bifocal RoPE attention
-// (sm_100a, bf16, head_dim 128, up to 8 query heads per kv head).
+// (sm_100a, bf16, head_dim 64 or 128, up to 8 query heads per kv head).
 //
 // One generation step against a standard-RoPE cache that is never rewritten
 // (Jet-Long technical summary, §2 "Rotação de Correção On-the-Fly"): local
@@ -642,7 +642,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
 // Split plan: one CTA per SM (the rings take ~200 KB of shared memory), one
 // wave of 148, whole 128-key tiles.
 void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk) {
-  const int ns0 = max(1, 148 / max(1, batch * Hkv));
+  const long long bh = (long long)batch * (long long)Hkv;
+  const int ns0 = bh >= 148 ? 1 : (int)(148 / max(1LL, bh));
   const int maxL = max(1, max_seqlen);
   int c = (maxL + ns0 - 1) / ns0;
   c = (c + dtc::TK - 1) / dtc::TK * dtc::TK;

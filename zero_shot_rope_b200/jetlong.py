@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
     L.jl_bifocal_decode_noalloc.restype = ctypes.c_int
     L.jl_bifocal_decode_noalloc.argtypes = [c_p, c_p, c_p, c_p, c_i32, c_i32, c_i32, c_i32, c_i32, c_i32,
                                             c_i64, c_i32, c_d, c_p, c_p, ctypes.c_int, c_u32, c_p]
+    L.jl_bifocal_decode_noalloc_error.restype = ctypes.c_int
+    L.jl_bifocal_decode_noalloc_error.argtypes = [ctypes.POINTER(c_i32), c_p]
     _lib = L
     return L
 
@@ -229,3 +231,13 @@ def jl_bifocal_decode_noalloc(q, k_cache, v_cache, seqlens, max_seqlen, w_pretra
                                            float(rope_theta), _ptr(out), _ptr(lse), _dtype_code(q), int(flags),
                                            _stream(stream)))
     return out, lse
+
+
+def jl_bifocal_decode_noalloc_error(stream=None) -> int:
+    """The kernel error word of the last jl_bifocal_decode_noalloc call (0: no
+    error).  Enqueues the copy on ``stream`` and synchronises it."""
+    word = ctypes.c_int32(-1)
+    st = _stream(stream)
+    _check(lib().jl_bifocal_decode_noalloc_error(ctypes.byref(word), st))
+    (stream or torch.cuda.current_stream()).synchronize()
+    return int(word.value)
