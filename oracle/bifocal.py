@@ -7,7 +7,7 @@ Every function follows a passage of the paper's technical summary
 ("Resumo Técnico: Jet-Long", gist.science, Portuguese; the French "Résumé
 Technique : Jet-Long" repeats it).  Section names below are that page's.
 
-Readings where the pages leave a step open (each also listed in the design doc):
+Readings where the pages leave a step open:
 
 * local window: key j is local for query i iff 0 <= p_i - p_j < w0, i.e. the
   window holds w0 keys including the query's own position;

@@ -47,9 +47,10 @@ def prefill_gpu(q, k, v, cu, w_pre, w0, theta, flags=0, with_lse=True):
     return out, lse
 
 
-def sample_rows(lengths, w0, G_list, n_random=48, seed=0):
-    """Stratified sample of global rows: first/last rows of every sequence,
-    rows around w0, around multiples of G and of the 128-row tile, and seeded
+def sample_rows(lengths, w0, G_list, n_edge=256, n_random=512, seed=0):
+    """Stratified sample of global rows, per sequence: the first and last
+    ``n_edge`` rows, rows around w0, around the first multiples of G and of
+    the 128-row tile, around the quarter points, and ``n_random`` seeded
     random rows."""
     rng = np.random.default_rng(seed)
     rows = set()
@@ -57,12 +58,10 @@ def sample_rows(lengths, w0, G_list, n_random=48, seed=0):
     for L, G in zip(lengths, G_list):
         if L == 0:
             continue
-        local = set(range(min(L, 24))) | set(range(max(0, L - 24), L))
-        for c in (w0 - 1, w0, w0 + 1, 127, 128, 129, L // 2, L // 2 + 1, 4 * G - 1, 4 * G):
-            if 0 <= c < L:
-                local.add(c)
-        for t in range(1, 4):
-            c = (L // 4) * t
+        local = set(range(min(L, n_edge))) | set(range(max(0, L - n_edge), L))
+        marks = [w0, 128, 256, L // 2] + [m * G for m in (1, 2, 3, 4, 1000)] + [(L // 4) * t for t in (1, 2, 3)]
+        marks += [128 * m for m in (33, 100, 511)]
+        for c in marks:
             for d in (-1, 0, 1):
                 if 0 <= c + d < L:
                     local.add(c + d)
@@ -70,3 +69,19 @@ def sample_rows(lengths, w0, G_list, n_random=48, seed=0):
         rows |= {start + r for r in local}
         start += L
     return np.array(sorted(rows), dtype=np.int64)
+
+
+def oracle_rows_threaded(fn, rows, *args, threads=None, **kw):
+    """Evaluate the prefill oracle ``fn(*args, rows=part, **kw)`` on parts of
+    ``rows`` in a pool of threads (NumPy releases the GIL in its large array
+    operations; one BLAS thread each) and reassemble (out, lse)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    from threadpoolctl import threadpool_limits
+
+    n = threads or max(1, min(32, (os.cpu_count() or 2) - 1))
+    parts = [p for p in np.array_split(np.asarray(rows), min(n, max(1, len(rows) // 32))) if len(p)]
+    with threadpool_limits(1), ThreadPoolExecutor(len(parts)) as ex:
+        res = list(ex.map(lambda part: fn(*args, rows=part, **kw), parts))
+    return np.concatenate([r[0] for r in res], axis=0), np.concatenate([r[1] for r in res], axis=1)
