@@ -279,7 +279,7 @@ def run_ours(args, world, rank, local):
     pre_ms_max = max_over_ranks(sum(pre_ms), world, dev)
     dec_ms_max = max_over_ranks(sum(dec_ms), world, dev)
     value = world * args.steps * pf_flops / (pre_ms_max * 1e-3) / 1e12
-    launches_per_step = 2 + 2 * n_dec  # prefill: pre-rotation + attention; decode: partial + combine
+    launches_per_step = 1 + 2 * n_dec  # prefill: attention; decode: partial + combine
 
     # ---- plain-causal comparison (outside the timed region): bifocal and
     # plain steps alternate so both see the same clocks (a long step runs
@@ -385,7 +385,7 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"replicas x{world}", "l2": "inputs larger than L2 (no flush needed)"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": kernel_traffic("bifocal_prefill2_kernel"),
-                     "kernel": "jl_bifocal_prefill (K pre-rotation + bifocal_prefill2_kernel, two heads per CTA)",
+                     "kernel": "bifocal_prefill2_kernel (two heads per CTA, in-tile key correction)",
                      "peak_kind": f"{peak_kind} bf16 sustained",
                      "frac_of_burst_peak": achieved / peaks["bf16_tflops"]},
         "decode": {"us_per_tok": dec_us_tok, "hbm_gbs": dec_gbs, "hbm_peak_gbs": peaks["hbm_gbs"],
@@ -405,6 +405,126 @@ def run_ours(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def _median_ms(fn, reps):
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def _case_inputs(args, dev):
+    seqlens = tuple(args.seqlens) if args.seqlens else (args.seqlen,)
+    q, k, v, cu = synth.random_case(3, seqlens, args.hq, args.hkv, args.head_dim, torch.bfloat16)
+    return seqlens, q.to(dev), k.to(dev), v.to(dev), cu.to(dev)
+
+
+def run_case(args):
+    """--only: run one call --reps times through the C ABI (a profiler driver:
+    the first call is a warm-up to skip with ``ncu -s``), then print its
+    median time."""
+    from zero_shot_rope_b200 import build
+    from zero_shot_rope_b200 import jetlong as jl
+
+    build.build()
+    dev = torch.device("cuda:0")
+    flags = (jl.JL_FLAG_PLAIN_CAUSAL if args.plain else 0) | (jl.JL_FLAG_PREROTATE_K if args.prerotate else 0)
+    D = args.head_dim
+    if args.only in ("prefill", "chunk"):
+        seqlens, q, k, v, cu = _case_inputs(args, dev)
+        if args.only == "prefill":
+            out = torch.empty_like(q)
+            ws = torch.zeros(jl.jl_bifocal_prefill_workspace_size(len(seqlens), q.shape[0], args.hq, args.hkv, D,
+                                                                  torch.bfloat16, flags), dtype=torch.uint8, device=dev)
+            fn = lambda: jl.jl_bifocal_prefill(q, k, v, cu, max(seqlens), args.w_pre, args.w0, 1e6, out=out,  # noqa
+                                               flags=flags, workspace=ws)
+            flops = sum(4.0 * D * args.hq * L * (L + 1) / 2 for L in seqlens)
+        else:
+            L, n = seqlens[0], args.chunk
+            qc = q[L - n:].contiguous()
+            out = torch.empty_like(qc)
+            cuq = torch.tensor([0, n], dtype=torch.int32, device=dev)
+            ws = torch.zeros(jl.jl_bifocal_prefill_workspace_size(1, L, args.hq, args.hkv, D, torch.bfloat16, flags),
+                             dtype=torch.uint8, device=dev)
+            fn = lambda: jl.jl_bifocal_prefill_kv(qc, k, v, cuq, cu, n, args.w_pre, args.w0, 1e6, out=out,  # noqa
+                                                  flags=flags, workspace=ws)
+            flops = sum(4.0 * D * args.hq * (L - n + i + 1) for i in range(n))
+        for _ in range(args.reps):
+            fn()
+        torch.cuda.synchronize()
+        ms = _median_ms(fn, 3) if args.time else None
+        print(json.dumps({"case": args.only, "seqlens": list(seqlens), "heads": f"{args.hq}/{args.hkv}",
+                          "head_dim": D, "flags": flags, "error_word": int(ws[:4].view(torch.int32).item()),
+                          "ms": ms, "tflops": flops / ms / 1e9 if ms else None}), flush=True)
+    else:
+        g = torch.Generator().manual_seed(5)
+        cap = args.seqlen
+        kc = torch.randn(1, cap, args.hkv, D, generator=g).to(torch.bfloat16).to(dev)
+        vc = torch.randn(1, cap, args.hkv, D, generator=g).to(torch.bfloat16).to(dev)
+        qd = torch.randn(1, args.hq, D, generator=g).to(torch.bfloat16).to(dev)
+        sl = torch.tensor([cap], dtype=torch.int32, device=dev)
+        out = torch.empty_like(qd)
+        ws = torch.zeros(jl.jl_bifocal_decode_workspace_size(1, args.hq, args.hkv, D, cap), dtype=torch.uint8,
+                         device=dev)
+        fn = lambda: jl.jl_bifocal_decode(qd, kc, vc, sl, cap, args.w_pre, args.w0, 1e6, out=out,  # noqa
+                                          flags=flags & jl.JL_FLAG_PLAIN_CAUSAL, workspace=ws)
+        for _ in range(args.reps):
+            fn()
+        torch.cuda.synchronize()
+        us = _median_ms(lambda: [fn() for _ in range(20)], 3) * 1e3 / 20 if args.time else None
+        print(json.dumps({"case": "decode", "L": cap, "heads": f"{args.hq}/{args.hkv}", "head_dim": D,
+                          "flags": flags, "us_per_call": us,
+                          "gbs": 2 * cap * args.hkv * D * 2 / us / 1e3 if us else None}), flush=True)
+
+
+def run_sweep_w0(args):
+    """--sweep-w0: prefill TFLOP/s and decode us/token across local-window
+    sizes, each beside the plain-causal call on the same inputs (markdown)."""
+    from zero_shot_rope_b200 import build
+    from zero_shot_rope_b200 import jetlong as jl
+
+    build.build()
+    dev = torch.device("cuda:0")
+    L, Hq, Hkv, D = args.seqlen, args.hq, args.hkv, args.head_dim
+    _, q, k, v, cu = _case_inputs(args, dev)
+    out = torch.empty_like(q)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    flops = 4.0 * D * Hq * L * (L + 1) / 2
+    kc, vc = k.view(1, L, Hkv, D), v.view(1, L, Hkv, D)
+    qd = q[L - 1:L].contiguous()
+    od = torch.empty_like(qd)
+    sl = torch.tensor([L], dtype=torch.int32, device=dev)
+    wsd = torch.zeros(jl.jl_bifocal_decode_workspace_size(1, Hq, Hkv, D, L), dtype=torch.uint8, device=dev)
+    G = jl.jl_group_size(L, args.w_pre)
+
+    def prefill(w0, flags):
+        return lambda: jl.jl_bifocal_prefill(q, k, v, cu, L, args.w_pre, w0, 1e6, out=out, flags=flags,
+                                             workspace=ws)
+
+    def decode(w0, flags, n=20):
+        return lambda: [jl.jl_bifocal_decode(qd, kc, vc, sl, L, args.w_pre, w0, 1e6, out=od, flags=flags,
+                                             workspace=wsd) for _ in range(n)]
+
+    plain_ms = _median_ms(prefill(0, jl.JL_FLAG_PLAIN_CAUSAL), args.reps)
+    plain_us = _median_ms(decode(0, jl.JL_FLAG_PLAIN_CAUSAL), args.reps) * 1e3 / 20
+    print(f"L = {L}, {Hq}/{Hkv} heads, D = {D}, w_pre = {args.w_pre} (G = {G}), bf16")
+    print()
+    print("| w0 | prefill ms | prefill TFLOP/s | vs plain | decode us/token | vs plain |")
+    print("|---:|---:|---:|---:|---:|---:|")
+    print(f"| plain | {plain_ms:.2f} | {flops / plain_ms / 1e9:.1f} | 1.000 | {plain_us:.1f} | 1.000 |")
+    for w0 in args.sweep_w0:
+        ms = _median_ms(prefill(w0, 0), args.reps)
+        us = _median_ms(decode(w0, 0), args.reps) * 1e3 / 20
+        print(f"| {w0} | {ms:.2f} | {flops / ms / 1e9:.1f} | {ms / plain_ms:.3f} | {us:.1f} | {us / plain_us:.3f} |",
+              flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -416,7 +536,29 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the extra workloads after the timed region")
+    # one call, for profilers (--only) and the w0 sweep (--sweep-w0)
+    ap.add_argument("--only", choices=["prefill", "chunk", "decode"])
+    ap.add_argument("--sweep-w0", type=int, nargs="+")
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--time", action="store_true", help="--only: also print the median time of 3 more calls")
+    ap.add_argument("--seqlen", type=int, default=32768)
+    ap.add_argument("--seqlens", type=int, nargs="+", help="--only prefill: packed sequence lengths")
+    ap.add_argument("--chunk", type=int, default=512, help="--only chunk: new tokens at the end of --seqlen")
+    ap.add_argument("--hq", type=int, default=32)
+    ap.add_argument("--hkv", type=int, default=8)
+    ap.add_argument("--head-dim", type=int, default=128)
+    ap.add_argument("--w-pre", type=int, default=32768)
+    ap.add_argument("--w0", type=int, default=4096)
+    ap.add_argument("--plain", action="store_true")
+    ap.add_argument("--prerotate", action="store_true", help="ablation: grouped keys from a pre-pass")
     args = ap.parse_args()
+    if args.only:
+        run_case(args)
+        return
+    if args.sweep_w0:
+        run_sweep_w0(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()

@@ -65,6 +65,12 @@ typedef enum {
                                      the comparison mode (G forced to 1)      */
 #define JL_FLAG_SIMT 0x2u         /* prefill: run the SIMT reference kernel
                                      instead of the tensor-core kernel       */
+#define JL_FLAG_PREROTATE_K 0x4u  /* prefill, ablation of the in-tile key
+                                     correction: a pre-pass writes the
+                                     grouped keys R(f(j)-j) K~ of every key
+                                     into the workspace (size it with this
+                                     flag) and the grouped visits load them;
+                                     same result, more HBM traffic           */
 
 /* Human-readable name of a status code (static string). */
 const char *jl_status_string(jl_status s);

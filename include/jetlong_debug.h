@@ -23,6 +23,8 @@
 #ifndef JETLONG_DEBUG_H
 #define JETLONG_DEBUG_H
 
+#include <stdint.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -41,6 +43,26 @@ int jl_debug_prefill_visits(int L, int Lk, int w0, int window, int G, int qt, in
  */
 int jl_debug_decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int window, int bf16,
                          int *nsplit, int *chunk, long long *partial_rows);
+
+/*
+ * jl_debug_set_wait_limit — the time limit, in nanoseconds, of the kernels'
+ * bounded pipeline waits on the current device (0 restores the default of
+ * 2 s).  A wait that runs out sets a bit of the call's error word, stops the
+ * kernel's other roles, lets its own copies and tensor-core work finish and
+ * returns; the call's output is then not valid.  Shortening the limit lets a
+ * test make such a wait run out without withholding any work: nothing faults
+ * and the context stays usable.  The waits that let a CTA's own copies land
+ * before it exits keep their fixed limit.  Synchronous (cudaMemcpyToSymbol);
+ * returns 0, or -1 with jl_last_error() set.
+ */
+int jl_debug_set_wait_limit(unsigned long long ns);
+
+/*
+ * jl_debug_angle_cs — the kernels' correction angle on the host: cos and sin
+ * of n * inv_freq, evaluated in fp64 by the kernels' own call-free sine and
+ * cosine and rounded to fp32.  Host-only; no CUDA call.
+ */
+void jl_debug_angle_cs(int32_t n, double inv_freq, float *c, float *s);
 
 #ifdef __cplusplus
 }

@@ -143,7 +143,11 @@ def test_workspace_sizes_are_consistent():
     assert big >= small > 0
     import torch
     assert jl.jl_bifocal_prefill_workspace_size(1, 1024, 2, 1, 64, torch.float32) == 0
-    assert jl.jl_bifocal_prefill_workspace_size(1, 1024, 32, 8, 128, torch.bfloat16) >= 1024 * 8 * 128 * 2
+    # the product path needs only the 256-byte error word; the pre-rotation
+    # ablation also holds the grouped keys (one K-sized buffer)
+    assert jl.jl_bifocal_prefill_workspace_size(1, 1024, 32, 8, 128, torch.bfloat16) == 256
+    assert jl.jl_bifocal_prefill_workspace_size(1, 1024, 32, 8, 128, torch.bfloat16,
+                                                jl.JL_FLAG_PREROTATE_K) >= 256 + 1024 * 8 * 128 * 2
 
 
 def _prefill_kv_raw(jl, **kw):

@@ -36,11 +36,13 @@ CASES = [
 
 
 @pytest.mark.parametrize("seqlens,Hq,Hkv,w_pre,w0", CASES)
-@pytest.mark.parametrize("kernel", ["tensor", "simt"])
+@pytest.mark.parametrize("kernel", ["tensor", "prerotated", "simt"])
 def test_bf16_cases_full(seqlens, Hq, Hkv, w_pre, w0, kernel):
+    # "tensor": grouped keys rotated in the tile (the product path);
+    # "prerotated": the ablation that writes them in a pre-pass
     J = jl()
     q, k, v, cu = synth.random_case(sum(seqlens) + 7 * Hq + w0, seqlens, Hq, Hkv, 128, torch.bfloat16)
-    flags = J.JL_FLAG_SIMT if kernel == "simt" else 0
+    flags = {"tensor": 0, "prerotated": J.JL_FLAG_PREROTATE_K, "simt": J.JL_FLAG_SIMT}[kernel]
     out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e6, flags=flags)
     ro, rl = oracle.bifocal_attention(q, k, v, cu, w_pre, w0, 1e6)
     assert_close(to_np(out), ro, torch.bfloat16, "out")
@@ -82,14 +84,20 @@ def test_tensor_kernel_matches_simt_kernel():
     assert_close(to_np(a)[np.arange(0, 3000, 97)], ro, torch.bfloat16, "tensor vs oracle")
 
 
-def test_kernel_error_word_stays_clear():
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (3, 1)])
+def test_kernel_error_word_stays_clear_in_a_256_byte_workspace(Hq, Hkv):
+    # the in-tile key correction needs no K-sized scratch: the default
+    # workspace is the 256-byte error word alone
     J = jl()
-    q, k, v, cu = synth.random_case(3, (1000,), 4, 2, 128, torch.bfloat16)
+    q, k, v, cu = synth.random_case(3, (1000,), Hq, Hkv, 128, torch.bfloat16)
     dev = torch.device("cuda:0")
-    ws = torch.zeros(J.jl_bifocal_prefill_workspace_size(1, 1000, 4, 2, 128), dtype=torch.uint8, device=dev)
-    J.jl_bifocal_prefill(q.to(dev), k.to(dev), v.to(dev), cu.to(dev), 1000, 300, 200, 1e6, workspace=ws)
+    assert J.jl_bifocal_prefill_workspace_size(1, 1000, Hq, Hkv, 128) == 256
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    out, _ = J.jl_bifocal_prefill(q.to(dev), k.to(dev), v.to(dev), cu.to(dev), 1000, 300, 200, 1e6, workspace=ws)
     torch.cuda.synchronize()
     assert int(ws[:4].view(torch.int32).item()) == 0
+    ro, _ = oracle.bifocal_attention(q, k, v, cu, 300, 200, 1e6, rows=np.arange(0, 1000, 37))
+    assert_close(to_np(out)[np.arange(0, 1000, 37)], ro, torch.bfloat16, "out")
 
 
 @pytest.mark.parametrize("name", ["prefill_32k_g1", "prefill_128k_g4", "varlen_4seq"])
@@ -180,9 +188,11 @@ D64_CASES = [
 
 
 @pytest.mark.parametrize("seqlens,Hq,Hkv,w_pre,w0", D64_CASES)
-def test_head_dim_64_bf16_full(seqlens, Hq, Hkv, w_pre, w0):
+@pytest.mark.parametrize("prerotated", [False, True])
+def test_head_dim_64_bf16_full(seqlens, Hq, Hkv, w_pre, w0, prerotated):
+    J = jl()
     q, k, v, cu = synth.random_case(sum(seqlens) + 64 + w0, seqlens, Hq, Hkv, 64, torch.bfloat16)
-    out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e4)
+    out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e4, flags=J.JL_FLAG_PREROTATE_K if prerotated else 0)
     ro, rl = oracle.bifocal_attention(q, k, v, cu, w_pre, w0, 1e4)
     assert_close(to_np(out), ro, torch.bfloat16, "out")
     assert_close(to_np(lse), rl, torch.bfloat16, "lse")

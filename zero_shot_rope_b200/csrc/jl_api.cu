@@ -144,7 +144,7 @@ jl_status jl_bifocal_prefill_kv(const void *q, const void *k, const void *v, voi
   if ((s = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return s;
   if (window < 0) return fail(JL_ERR_INVALID_ARG, "window must be >= 0 (0: no window), got %d", window);
   if (dtype != JL_BF16 && dtype != JL_FP32) return fail(JL_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
-  if (flags & ~(uint32_t)(JL_FLAG_PLAIN_CAUSAL | JL_FLAG_SIMT))
+  if (flags & ~(uint32_t)(JL_FLAG_PLAIN_CAUSAL | JL_FLAG_SIMT | JL_FLAG_PREROTATE_K))
     return fail(JL_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
   if (batch < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0)
     return fail(JL_ERR_INVALID_ARG, "batch, token counts and max_seqlen must be >= 0");
@@ -266,3 +266,26 @@ jl_status jl_bifocal_decode(const void *q, const void *k_cache, const void *v_ca
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- test hooks
+namespace jl {
+cudaError_t set_wait_limit_prefill(unsigned long long ns);
+cudaError_t set_wait_limit_decode_tc(unsigned long long ns);
+cudaError_t set_wait_limit_decode(unsigned long long ns);
+}  // namespace jl
+
+extern "C" int jl_debug_set_wait_limit(unsigned long long ns) {
+  if (ns == 0) ns = 2000000000ull;
+  cudaError_t e = jl::set_wait_limit_prefill(ns);
+  if (e == cudaSuccess) e = jl::set_wait_limit_decode_tc(ns);
+  if (e == cudaSuccess) e = jl::set_wait_limit_decode(ns);
+  if (e != cudaSuccess) {
+    fail(JL_ERR_CUDA, "setting the wait limit failed: %s", cudaGetErrorString(e));
+    return -1;
+  }
+  return 0;
+}
+
+extern "C" void jl_debug_angle_cs(int32_t n, double inv_freq, float *c, float *s) {
+  jl::angle_cs(n, inv_freq, *c, *s);
+}

@@ -31,11 +31,52 @@ __host__ __device__ __forceinline__ int32_t fmap(int32_t x, int32_t G) { return 
 // n(p) = p - f(p) >= 0: the correction rotates by -n(p) positions.
 __host__ __device__ __forceinline__ int32_t corr_n(int32_t p, int32_t G) { return p - p / G; }
 
+// sin and cos of an fp64 angle x, |x| < 2^40, with no function call (so it
+// may run inside kernels that rebalance registers with setmaxnreg, where
+// ptxas cannot handle calls).  Cody–Waite reduction by pi/2: k = rint(x 2/pi)
+// and r = x - k pi/2 in two fused multiply-adds against pi/2 written as the
+// sum of two doubles, exact to ~1e-16 for every k < 2^53; then the Taylor
+// series of sin (to r^17) and cos (to r^16) on |r| <= pi/4, whose truncation
+// errors are below 1e-19; then the quadrant k mod 4.
+__host__ __device__ __forceinline__ void sincos_fp64(double x, double &sn, double &cs) {
+  const double two_over_pi = 0.63661977236758134308;
+  const double pio2_hi = 1.5707963267948966192;     // fp64 nearest to pi/2
+  const double pio2_lo = 6.1232339957367660359e-17;  // pi/2 - pio2_hi
+  const double k = rint(x * two_over_pi);
+  double r = fma(-k, pio2_hi, x);
+  r = fma(-k, pio2_lo, r);
+  const double r2 = r * r;
+  double ps = 1.0 / 355687428096000.0;  // 1/17!
+  ps = fma(ps, -r2, 1.0 / 1307674368000.0);
+  ps = fma(ps, -r2, 1.0 / 6227020800.0);
+  ps = fma(ps, -r2, 1.0 / 39916800.0);
+  ps = fma(ps, -r2, 1.0 / 362880.0);
+  ps = fma(ps, -r2, 1.0 / 5040.0);
+  ps = fma(ps, -r2, 1.0 / 120.0);
+  ps = fma(ps, -r2, 1.0 / 6.0);
+  const double sr = fma(-r * r2, ps, r);  // r - r^3/3! + r^5/5! - ...
+  double pc = 1.0 / 20922789888000.0;   // 1/16!
+  pc = fma(pc, -r2, 1.0 / 87178291200.0);
+  pc = fma(pc, -r2, 1.0 / 479001600.0);
+  pc = fma(pc, -r2, 1.0 / 3628800.0);
+  pc = fma(pc, -r2, 1.0 / 40320.0);
+  pc = fma(pc, -r2, 1.0 / 720.0);
+  pc = fma(pc, -r2, 1.0 / 24.0);
+  pc = fma(pc, -r2, 1.0 / 2.0);
+  const double cr = fma(-r2, pc, 1.0);  // 1 - r^2/2! + r^4/4! - ...
+  switch ((long long)k & 3) {
+    case 0: sn = sr; cs = cr; break;
+    case 1: sn = cr; cs = -sr; break;
+    case 2: sn = -sr; cs = -cr; break;
+    default: sn = -cr; cs = sr; break;
+  }
+}
+
 // cos / sin of the angle n * invf, formed in fp64 from the exact integer n and
-// evaluated with the fp64 sincos before rounding to fp32.
-__device__ __forceinline__ void angle_cs(int32_t n, double invf, float &c, float &s) {
+// evaluated in fp64 before rounding to fp32.
+__host__ __device__ __forceinline__ void angle_cs(int32_t n, double invf, float &c, float &s) {
   double sd, cd;
-  sincos((double)n * invf, &sd, &cd);
+  sincos_fp64((double)n * invf, sd, cd);
   c = (float)cd;
   s = (float)sd;
 }

@@ -710,3 +710,10 @@ extern "C" int jl_debug_decode_plan(int batch, int Hq, int Hkv, int D, int max_s
   *partial_rows = (long long)jl::decode_partial_rows(batch, Hq, Hkv, D, max_seqlen);
   return 0;
 }
+
+namespace jl {
+// Test hook: the limit of the bounded waits of this file's kernels.
+cudaError_t set_wait_limit_decode(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
+}  // namespace jl

@@ -314,7 +314,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
           t_idle = gtime();
         } else if ((++spins & 31u) == 0) {
           if (abort_flag) ok = false;
-          else if (gtime() - t_idle > 2000000000ull) {
+          else if (gtime() - t_idle > *(volatile unsigned long long *)&g_wait_limit_ns) {
             abort_flag = 1;
             atomicOr(p.err, ERR_TIMEOUT);
             ok = false;
@@ -700,4 +700,11 @@ cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtenso
   return cudaGetLastError();
 }
 
+}  // namespace jl
+
+namespace jl {
+// Test hook: the limit of the bounded waits of this file's kernels.
+cudaError_t set_wait_limit_decode_tc(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
 }  // namespace jl

@@ -1,43 +1,40 @@
-// Tensor-core prefill kernel for Dynamic Bifocal RoPE attention (sm_100a).
+// Tensor-core prefill kernels for Dynamic Bifocal RoPE attention (sm_100a).
 //
 // Jet-Long technical summary, §2 "Mecanismos de Eficiência de Inferência":
 // the local window (base RoPE), the full causal pass over grouped queries and
 // keys, and the window pass over grouped queries and keys are merged by
 // inclusion–exclusion with LSE statistics, which gives the exact
-// distance-routed attention (§1 "Janela Local" / "Janela Remota").  This
-// kernel computes that exact value in one causal pass: every (query tile,
+// distance-routed attention (§1 "Janela Local" / "Janela Remota").  These
+// kernels compute that exact value in one causal pass: every (query tile,
 // key tile) pair is visited with the base operands where all its distances
 // are < w0, with the grouped operands where all are >= w0, and twice (once
 // each, complementary masks) on the tile that straddles d = w0; one online
 // softmax runs over all visits.
 //
-// Two kernels, both templated on the head_dim D (64 or 128):
-// bifocal_prefill2_kernel takes two query heads of one GQA group per CTA
-// (even groups; its layout is described above its definition), and
-// bifocal_prefill_kernel one head per CTA:
-//   warps 0-3  softmax / correction / epilogue: thread r owns query row r and
-//              TMEM lane r; also rotates the query tile into grouped
-//              positions once (R(f(i) - i), §2 "Rotação de Correção").
-//   warp 4     TMA producer of Q and K tiles (128 rows x D bf16, SWIZZLE_128B
-//              boxes of 64 columns).
-//   warp 5     TMEM allocator and the single-thread tcgen05.mma issuer:
-//              S = Q K^T (SS form) into a double-buffered TMEM S, then
-//              O += P V with P read from TMEM (TS form).
-//   warp 6     TMA producer of V tiles.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D) (fp32, lane = row);
-// P (bf16 pairs) overwrites the first 64 columns of its S buffer.
+// The grouped operands come from the on-the-fly correction rotation of §2
+// "Rotação de Correção On-the-Fly", applied in the kernels and never written
+// back: the query tile is rotated once per CTA by R(f(i) - i), and each key
+// tile of a grouped visit is rotated in place in shared memory by
+// R(f(j) - j), between its TMA load and its QK products, by a warpgroup of
+// its own (KeyCorrection below).
 //
-// The grouped keys K_g = R(f(j) - j) K~ are produced once per key by
-// prerotate_k_kernel; grouped visits load K_g tiles instead of K~ tiles.
+// Two kernels, both templated on the head_dim D (64 or 128), both organised
+// in whole warpgroups so that `setmaxnreg` can move registers from the
+// producer, MMA and rotation roles to the softmax warpgroups:
+//   bifocal_prefill2_kernel  two query heads of one GQA group per CTA (even
+//                            groups), 4 warpgroups; layout above its definition
+//   bifocal_prefill_kernel   one query head per CTA (odd groups), 3 warpgroups
 //
-// Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the kernel
-// records an error code, tells the other roles to stop, waits (bounded) for
-// its own copies and MMAs in flight, frees TMEM and returns.
+// Every mbarrier wait is bounded (%globaltimer); on expiry the kernel records
+// an error code, tells the other roles to stop, waits (bounded) for its own
+// copies and MMAs in flight, frees TMEM and returns.
 #include <cuda.h>
 
 #include <type_traits>
 
+#include "../../include/jetlong.h"
 #include "jl_common.cuh"
+#define JL_WAITS_INLINE 1  // these kernels use setmaxnreg: no calls
 #include "jl_ptx.cuh"
 
 namespace jl {
@@ -45,19 +42,26 @@ namespace tc {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
-constexpr int NKS = 2;   // K ring stages (one head per CTA)
+constexpr int P1_NKS = 3;  // K ring stages (one head per CTA)
 constexpr int NVS = 2;   // V ring stages (one head per CTA)
 constexpr int HALF_BYTES = BM * 64 * 2;  // one 64-column SWIZZLE_128B box of a 128-row tile
-constexpr int NUM_THREADS = 224;
 constexpr int OFF_Q = 0;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_O = 256;
 constexpr int HI_INF = 1 << 30;
 
+// one head per CTA: warpgroups softmax | producers + MMA | key correction
+constexpr int P1_THREADS = 384;
+constexpr uint32_t P1_REG_SOFTMAX = 232, P1_REG_IO = 104, P1_REG_KCORR = 168;  // 232 + 104 + 168 = 3 x 168
+// two heads per CTA: softmax A | softmax B | key correction | producers + MMA
+constexpr int P2_THREADS = 512;
+constexpr uint32_t P2_REG_SOFTMAX = 176, P2_REG_KCORR = 88, P2_REG_IO = 72;  // 2 x 176 + 88 + 72 = 4 x 128
+
 // error codes (bit flags) written to the workspace error word
 constexpr int ERR_TIMEOUT_PRODUCER = 1;
 constexpr int ERR_TIMEOUT_MMA = 2;
 constexpr int ERR_TIMEOUT_SOFTMAX = 4;
+constexpr int ERR_TIMEOUT_KCORR = 32;
 
 struct Params {
   const int32_t *cu;    // query prefix sums [batch + 1]
@@ -67,11 +71,21 @@ struct Params {
   long long w_pre;
   int w0, plain;
   int window;           // sliding-window width (0: none)
+  int kg_pre;           // 1: grouped keys were written by prerotate_k_kernel (ablation)
   __nv_bfloat16 *out;
   float *lse;
   int *err;
   float sl2;  // log2(e) / sqrt(D)
 };
+
+template <uint32_t R>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(R) : "memory");
+}
+template <uint32_t R>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(R) : "memory");
+}
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -145,23 +159,21 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 
-// Shared-memory matrix descriptors (tcgen05 format, version 1).
-// K-major, 128-byte swizzle: 8-row atoms of 128 B, atoms 1024 B apart.
-__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
-         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])
+               :
+               : "memory");
 }
-// MN-major, 128-byte swizzle: 64 contiguous N elements per 128 B row, 8 K rows
-// per 1024 B atom (SBO), N blocks of 64 `lbo` bytes apart.
-__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
-}
-// Instruction descriptor, kind::f16: D fp32, A/B bf16, M = 128, N = 128.
-constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 16);  // B (= V) is MN-major
 
-constexpr int P2_THREADS = 320;
 constexpr int P2_NKS = 3;
 constexpr int P2_NVS = 2;
 constexpr int P2_OFF_Q = 0;  // Q_A, Q_B
@@ -181,12 +193,28 @@ struct Geo {
   // one head per CTA: Q, Q_g, the K ring, the V ring
   static constexpr int P1_OFF_QG = TB;
   static constexpr int P1_OFF_K = 2 * TB;
-  static constexpr int P1_OFF_V = P1_OFF_K + NKS * TB;
+  static constexpr int P1_OFF_V = P1_OFF_K + P1_NKS * TB;
   static constexpr int P1_SMEM_ALLOC = P1_OFF_V + NVS * TB + 1024;
   // kind::f16, D fp32, A/B bf16, M = 128, N = D, B (= V) MN-major
   static constexpr uint32_t IDESC_PV =
       (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(D >> 3) << 17) | ((128u >> 4) << 24);
 };
+
+// Shared-memory matrix descriptors (tcgen05 format, version 1).
+// K-major, 128-byte swizzle: 8-row atoms of 128 B, atoms 1024 B apart.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// MN-major, 128-byte swizzle: 64 contiguous N elements per 128 B row, 8 K rows
+// per 1024 B atom (SBO), N blocks of 64 `lbo` bytes apart.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, M = 128, N = 128.
+constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t IDESC_PV = IDESC_QK | (1u << 16);  // B (= V) is MN-major
 
 // --------------------------------------------------------- tile schedule
 // A query tile: rows i0..i1 of a sequence with L queries at positions
@@ -265,22 +293,205 @@ __host__ __device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan
   }
 }
 
-// ----------------------------------------------------------------- kernel
+// ------------------------------------------------------------ key correction
+// §2 "Rotação de Correção On-the-Fly": the grouped branch scores a remote key
+// at its grouped position, K_g = R(f(j) - j) K~ = R(-n(j)) K~ with
+// n(j) = j - floor(j / G), while the stored keys stay as they are.  One
+// warpgroup of the prefill CTA applies that rotation in place to the K tile
+// of every grouped visit, in shared memory, after the tile's TMA load and
+// before its QK products read it.
+//
+// Thread t (0..127) owns the 8 pairs k = 8 lc .. 8 lc + 7 (pair k: elements k
+// and k + D/2) of RPT consecutive rows r0 .. r0 + RPT - 1 of every tile:
+//   D = 128: lc = t % 8, rows 8 (t / 8) ..; element k in box 0 and k + 64 in
+//            the same 16-byte chunk of box 1;
+//   D = 64:  lc = t % 4, rows 4 (t / 4) ..; chunk lc pairs with chunk lc + 4
+//            of the same 128-byte row.
+// The eight lanes of each shared-memory phase touch eight distinct 16-byte
+// bank groups in both layouts.  From one key to the next, n grows by one
+// except where the next key index is a multiple of G, so along its rows a
+// thread steps its rotation by R(1) or keeps it.  The rotation of its first
+// row advances once per tile by R(delta), delta = n(j + BN) - n(j): with
+// BN = b G + sigma and rho = j mod G, delta = BN - b - [rho + sigma >= G], so
+// the step is R(BN - b), tabulated per CTA, times R(-1) when the carry is
+// set.  Angles are seeded in fp64 (the fp64 sine and cosine of the exact
+// integer multiple) and carried in fp32; a CTA advances at most L / BN tile
+// steps.
+struct KCorrTable {
+  float4 v[4][8];  // R(BN - b) per chunk lc: [cos 0-3, cos 4-7, sin 0-3, sin 4-7][lc]
+};
+
+__device__ __forceinline__ float2 bf2_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_bf2(float2 f) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(f.x, f.y);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+// (c, s) <- (c, s) x (c1, s1): rotation angles add
+__device__ __forceinline__ void compose2(float2 &c, float2 &s, float2 c1, float2 s1) {
+  const float2 cn = __ffma2_rn(c, c1, __fmul2_rn(neg2(s), s1));
+  const float2 sn = __ffma2_rn(s, c1, __fmul2_rn(c, s1));
+  c = cn;
+  s = sn;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 x;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(a));
+  return x;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 x) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
+               : "memory");
+}
+
+template <int D, int NSTAGE>
+struct KeyCorrection {
+  static constexpr int CPR = D / 16;          // 8-pair chunks per row
+  static constexpr int RPT = BN * CPR / 128;  // rows per thread per tile
+  int lc, r0, G, sigma, rho;
+  float2 bc[4], bs[4];  // rotation by n of the thread's first row, pairs (2w, 2w + 1) packed
+  float2 c1[4], s1[4];  // R(1)
+
+  // Set-up once per CTA, by all 128 threads of the warpgroup: R(BN - b) into
+  // `tab` (then a named barrier over the warpgroup), R(1) and the first
+  // tile's rotation in registers.  j_first: the first key of the first
+  // grouped visit.
+  __device__ __forceinline__ void init(int t, int j_first, int G_, const InvFreq &inv, KCorrTable &tab,
+                                       int bar_id) {
+    G = G_;
+    lc = t % CPR;
+    r0 = (t / CPR) * RPT;
+    sigma = BN % G;
+    if (t < 4 * CPR) {  // entry (j, chunk): four cos or sin values of one chunk
+      const int j = t / CPR, ch = t % CPR;
+      float cs[4], sn[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) angle_cs(BN - BN / G, inv.v[8 * ch + 4 * (j & 1) + e], cs[e], sn[e]);
+      tab.v[j][ch] = j < 2 ? make_float4(cs[0], cs[1], cs[2], cs[3]) : make_float4(sn[0], sn[1], sn[2], sn[3]);
+    }
+    const int J = j_first + r0;
+    rho = J % G;
+    const int n0 = corr_n(J, G);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      float ca, sa, cb, sb;
+      angle_cs(n0, inv.v[8 * lc + 2 * w], ca, sa);
+      angle_cs(n0, inv.v[8 * lc + 2 * w + 1], cb, sb);
+      bc[w] = make_float2(ca, cb);
+      bs[w] = make_float2(sa, sb);
+      angle_cs(1, inv.v[8 * lc + 2 * w], ca, sa);
+      angle_cs(1, inv.v[8 * lc + 2 * w + 1], cb, sb);
+      c1[w] = make_float2(ca, cb);
+      s1[w] = make_float2(sa, sb);
+    }
+    asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
+  }
+
+  // Rotate this thread's rows of one K tile (shared address of its first
+  // byte), then advance the first-row rotation to the next key tile.
+  __device__ __forceinline__ void rotate_tile(uint32_t tile, const KCorrTable &tab) {
+    float2 c[4], s[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      c[w] = bc[w];
+      s[w] = bs[w];
+    }
+    int rr = rho;  // key index of the current row, mod G
+#pragma unroll 1
+    for (int m = 0; m < RPT; ++m) {
+      const int row = r0 + m;
+      const int sw = row & 7;
+      const uint32_t pa = tile + row * 128 + ((lc ^ sw) << 4);
+      const uint32_t pb = D == 128 ? pa + HALF_BYTES : tile + row * 128 + (((lc + 4) ^ sw) << 4);
+      uint4 xa = lds128(pa), xb = lds128(pb);
+      uint32_t *ua = reinterpret_cast<uint32_t *>(&xa), *ub = reinterpret_cast<uint32_t *>(&xb);
+      // R(-n) (a, b) = (a cos + b sin, b cos - a sin)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float2 fa = bf2_f2(ua[w]), fb = bf2_f2(ub[w]);
+        ua[w] = f2_bf2(__ffma2_rn(fa, c[w], __fmul2_rn(fb, s[w])));
+        ub[w] = f2_bf2(__ffma2_rn(fb, c[w], __fmul2_rn(neg2(fa), s[w])));
+      }
+      sts128(pa, xa);
+      sts128(pb, xb);
+      if (m + 1 < RPT) {
+        if (rr + 1 == G) {
+          rr = 0;  // the next key starts a group: n unchanged
+        } else {
+          ++rr;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) compose2(c[w], s[w], c1[w], s1[w]);
+        }
+      }
+    }
+    // next tile: the first row advances by R(BN - b), and by R(-1) more when
+    // the key index's residue carries past G
+    const float4 tc0 = tab.v[0][lc], tc1 = tab.v[1][lc], ts0 = tab.v[2][lc], ts1 = tab.v[3][lc];
+    const float2 dc[4] = {make_float2(tc0.x, tc0.y), make_float2(tc0.z, tc0.w), make_float2(tc1.x, tc1.y),
+                          make_float2(tc1.z, tc1.w)};
+    const float2 ds[4] = {make_float2(ts0.x, ts0.y), make_float2(ts0.z, ts0.w), make_float2(ts1.x, ts1.y),
+                          make_float2(ts1.z, ts1.w)};
+    const bool carry = rho + sigma >= G;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      compose2(bc[w], bs[w], dc[w], ds[w]);
+      if (carry) compose2(bc[w], bs[w], c1[w], neg2(s1[w]));
+    }
+    rho += sigma - (carry ? G : 0);
+  }
+
+  // The role: for the grouped visits v = 0 .. n_grp - 1 (key tiles in
+  // ascending order, the first visits of the CTA), wait for the K tile of
+  // stage v % NSTAGE, rotate it, make the writes visible to the tensor core
+  // and release it to the MMA issuer.
+  __device__ __forceinline__ void run(int n_grp, uint32_t kring, int stage_bytes, uint64_t *bar_kf,
+                                      uint64_t *bar_kr, const KCorrTable &tab, volatile int *abort_flag,
+                                      int *err) {
+    for (int v = 0; v < n_grp; ++v) {
+      const int st = v % NSTAGE;
+      if (!__all_sync(0xffffffffu, wait_b(&bar_kf[st], (v / NSTAGE) & 1, abort_flag, err, ERR_TIMEOUT_KCORR)))
+        break;
+      rotate_tile(kring + st * stage_bytes, tab);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&bar_kr[st]);
+    }
+  }
+};
+
+// ------------------------------------------------------------------ kernels
+// One query head per CTA (odd GQA groups), 384 threads in 3 warpgroups:
+//   warps 0-3   softmax / correction / epilogue: thread r owns query row r and
+//               TMEM lane r; also rotates the query tile into grouped
+//               positions once (R(f(i) - i) into the Q_g buffer).
+//   warp 4      TMA producer of Q and K tiles (128 rows x D bf16, SWIZZLE_128B
+//               boxes of 64 columns).
+//   warp 5      TMEM allocator and the single-thread tcgen05.mma issuer:
+//               S = Q K^T (SS form) into a double-buffered TMEM S, then
+//               O += P V with P read from TMEM (TS form).
+//   warp 6      TMA producer of V tiles.   (warp 7 idle)
+//   warps 8-11  key correction: each grouped visit's K tile rotated in place.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D) (fp32, lane = row);
+// P (bf16 pairs) overwrites the first 64 columns of its S buffer.
 template <int D>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(P1_THREADS, 1)
 bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mK,
                        const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
                        const __grid_constant__ Params p, const __grid_constant__ InvFreq inv) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_qg, bar_kf[NKS], bar_ke[NKS], bar_vf[NVS], bar_ve[NVS],
-      bar_sf[2], bar_pr[2], bar_od, bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_qg, bar_kf[P1_NKS], bar_kr[P1_NKS], bar_ke[P1_NKS], bar_vf[NVS],
+      bar_ve[NVS], bar_sf[2], bar_pr[2], bar_od, bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ KCorrTable kctab;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work item (uniform across the CTA; invalid items exit before any barrier)
   using GG = Geo<D>;
+  constexpr int OFF_K1 = GG::P1_OFF_K;
+  constexpr int OFF_V1 = GG::P1_OFF_V;
   const int s = blockIdx.z, h = blockIdx.y;
   const int a = p.cu[s];                // first query token
   const int L = p.cu[s + 1] - a;        // queries
@@ -302,6 +513,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   const int kvh = h / (p.Hq / p.Hkv);
   const VisitPlan pl = make_plan(t, p.w0);
   const bool need_qg = pl.n_grp > 0;
+  const bool kcorr = need_qg && !p.kg_pre;  // grouped K tiles rotated in this CTA
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
@@ -309,7 +521,11 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   if (threadIdx.x == 0) {
     mbar_init(&bar_q, 1);
     mbar_init(&bar_qg, 128);
-    for (int i = 0; i < NKS; ++i) { mbar_init(&bar_kf[i], 1); mbar_init(&bar_ke[i], 1); }
+    for (int i = 0; i < P1_NKS; ++i) {
+      mbar_init(&bar_kf[i], 1);
+      mbar_init(&bar_kr[i], 128);
+      mbar_init(&bar_ke[i], 1);
+    }
     for (int i = 0; i < NVS; ++i) { mbar_init(&bar_vf[i], 1); mbar_init(&bar_ve[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&bar_sf[i], 1); mbar_init(&bar_pr[i], 128); }
     mbar_init(&bar_od, 1);
@@ -334,52 +550,57 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   const uint32_t tmem = tmem_slot;
 
   const int tok_q0 = a + t.i0;
-  if (warp == 4) {
-    // ================= producer: Q, then K tiles in visit order =================
-    if (lane == 0) {
+  if (warp >= 8) {
+    // ================= key correction (warps 8-11) =================
+    regs_dec<P1_REG_KCORR>();
+    if (kcorr) {
+      KeyCorrection<D, P1_NKS> kc;
+      kc.init(threadIdx.x - 256, pl.g_begin * BN, t.G, inv, kctab, 1);
+      kc.run(pl.n_grp, sbase + OFF_K1, GG::TB, bar_kf, bar_kr, kctab, &abort_flag, p.err);
+    }
+  } else if (warp >= 4) {
+    regs_dec<P1_REG_IO>();
+    if (warp == 4 && lane == 0) {
+      // ================= producer: Q, then K tiles in visit order =================
       mbar_expect_tx(&bar_q, GG::TB);
       for (int hf = 0; hf < GG::NH; ++hf) tma_load(&mQ, &bar_q, sbase + OFF_Q + hf * HALF_BYTES, 64 * hf, h, tok_q0);
       int v = 0;
-      bool ok = true;
       for (; v < pl.n_all; ++v) {
         int kt;
         Visit vx;
         visit_at(t, pl, p.w0, v, kt, vx);
-        const int st = v % NKS;
-        if (v >= NKS && !(ok = wait_b(&bar_ke[st], ((v / NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+        const int st = v % P1_NKS;
+        if (v >= P1_NKS &&
+            !wait_b(&bar_ke[st], ((v / P1_NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER))
           break;
-        const CUtensorMap *m = vx.grp ? &mKg : &mK;
-        const uint32_t dst = sbase + GG::P1_OFF_K + st * GG::TB;
+        const CUtensorMap *m = (vx.grp && p.kg_pre) ? &mKg : &mK;
+        const uint32_t dst = sbase + OFF_K1 + st * GG::TB;
         mbar_expect_tx(&bar_kf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
           tma_load(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
       }
       // drain: every load issued must land before the CTA may exit
-      for (int u = max(0, v - NKS); u < v; ++u) wait_drain(&bar_kf[u % NKS], (u / NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
+      for (int u = max(0, v - P1_NKS); u < v; ++u)
+        wait_drain(&bar_kf[u % P1_NKS], (u / P1_NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
       wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
-    }
-  } else if (warp == 6) {
-    // ================= producer: V tiles in visit order =================
-    if (lane == 0) {
+    } else if (warp == 6 && lane == 0) {
+      // ================= producer: V tiles in visit order =================
       int v = 0;
-      bool ok = true;
       for (; v < pl.n_all; ++v) {
         int kt;
         Visit vx;
         visit_at(t, pl, p.w0, v, kt, vx);
         const int st = v % NVS;
-        if (v >= NVS && !(ok = wait_b(&bar_ve[st], ((v / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
+        if (v >= NVS && !wait_b(&bar_ve[st], ((v / NVS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER))
           break;
-        const uint32_t dst = sbase + GG::P1_OFF_V + st * GG::TB;
+        const uint32_t dst = sbase + OFF_V1 + st * GG::TB;
         mbar_expect_tx(&bar_vf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
           tma_load(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
       }
       for (int u = max(0, v - NVS); u < v; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
-    }
-  } else if (warp == 5) {
-    // ================= MMA issuer (one thread) =================
-    if (lane == 0) {
+    } else if (warp == 5 && lane == 0) {
+      // ================= MMA issuer (one thread) =================
       bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
       bool qg_seen = false;
       int v = 0;
@@ -388,7 +609,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         if (!wait_b(&bar_vf[vs_], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         if (!wait_b(&bar_pr[u & 1], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t vaddr = sbase + GG::P1_OFF_V + vs_ * GG::TB;
+        const uint32_t vaddr = sbase + OFF_V1 + vs_ * GG::TB;
         const uint32_t pcol = tmem + (uint32_t)((u & 1) * 128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -402,26 +623,26 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         int kt;
         Visit vx;
         visit_at(t, pl, p.w0, v, kt, vx);
-        {
-          if (vx.grp && !qg_seen) {
-            if (!(ok = wait_b(&bar_qg, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
-            qg_seen = true;
-          }
-          const int st = v % NKS;
-          if (!(ok = wait_b(&bar_kf[st], (v / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
-          tc_fence_after();
-          const uint32_t qaddr = sbase + (vx.grp ? GG::P1_OFF_QG : OFF_Q);
-          const uint32_t kaddr = sbase + GG::P1_OFF_K + st * GG::TB;
-          const uint32_t scol = tmem + (uint32_t)((v & 1) * 128);
-#pragma unroll
-          for (int kk = 0; kk < GG::KSTEPS; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&bar_sf[v & 1]);
-          umma_commit(&bar_ke[st]);
-          if (v > 0 && !(ok = issue_pv(v - 1))) break;
+        if (vx.grp && !qg_seen) {
+          if (!(ok = wait_b(&bar_qg, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
+          qg_seen = true;
         }
+        const int st = v % P1_NKS;
+        // a grouped K tile is read once the key correction has rotated it
+        uint64_t *kready = (vx.grp && kcorr) ? &bar_kr[st] : &bar_kf[st];
+        if (!(ok = wait_b(kready, (v / P1_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
+        tc_fence_after();
+        const uint32_t qaddr = sbase + (vx.grp ? GG::P1_OFF_QG : OFF_Q);
+        const uint32_t kaddr = sbase + OFF_K1 + st * GG::TB;
+        const uint32_t scol = tmem + (uint32_t)((v & 1) * 128);
+#pragma unroll
+        for (int kk = 0; kk < GG::KSTEPS; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&bar_sf[v & 1]);
+        umma_commit(&bar_ke[st]);
+        if (v > 0 && !(ok = issue_pv(v - 1))) break;
       }
       if (ok && v > 0) issue_pv(v - 1);
       // all MMAs issued so far must finish before TMEM is released
@@ -430,6 +651,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     }
   } else {
     // ================= softmax warpgroup (warps 0-3) =================
+    regs_inc<P1_REG_SOFTMAX>();
     const int r = threadIdx.x;  // query row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int i = t.i0 + r;
@@ -609,8 +831,10 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
   }
 }
 
-// Grouped keys K_g = R(f(j) - j) K~ for every token of sequences with G > 1,
-// written once per key (all kv heads of a token share the angles).
+// Ablation of the key correction (JL_FLAG_PREROTATE_K): grouped keys
+// K_g = R(f(j) - j) K~ for every token of sequences with G > 1, written once
+// per key into the workspace (all kv heads of a token share the angles), and
+// TMA-loaded by the grouped visits instead of being rotated in the tile.
 __global__ void __launch_bounds__(256)
 prerotate_k_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ kg, int D,
                    const int32_t *__restrict__ cu, int batch, int T, int Hkv, long long w_pre,
@@ -676,12 +900,18 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // Two heads per CTA.
 //
 // The CTA takes one 128-row query tile of two query heads of the same GQA
-// group: both read the same K/V tiles (loaded once), and two softmax
-// warpgroups ping-pong against one MMA warp, so the tensor core always has
-// the other head's QK or PV to run while a softmax warpgroup works.
-//   warps 0-3 / 4-7  softmax of head A / head B (thread = row = TMEM lane)
-//   warp 8           TMA producers: lane 0 streams Q and K tiles, lane 1 V tiles
-//   warp 9           TMEM allocator and tcgen05.mma issuer
+// group: both read the same K/V tiles (loaded, and for grouped visits
+// rotated, once), and two softmax warpgroups ping-pong against one MMA warp,
+// so the tensor core always has the other head's QK or PV to run while a
+// softmax warpgroup works.  512 threads, 4 warpgroups:
+//   warps 0-3 / 4-7  softmax of head A / head B (thread = row = TMEM lane);
+//                    the row's 128 scores are read from TMEM once and stay
+//                    in registers (setmaxnreg gives these warpgroups the
+//                    registers the other two do not need)
+//   warps 8-11       key correction: each grouped visit's K tile rotated in
+//                    place, R(f(j) - j), before its QK products
+//   warp 12          TMA producers: lane 0 streams Q and K tiles, lane 1 V tiles
+//   warp 13          TMEM allocator and tcgen05.mma issuer   (warps 14-15 idle)
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [256+D,256+2D).
 // Visit order: every grouped visit (ascending key tile), then every base
 // visit.  The query tiles are rotated in place into grouped positions for
@@ -693,10 +923,11 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
                         const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
                         const __grid_constant__ Params p, const __grid_constant__ InvFreq inv) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_qg[2], bar_qfree, bar_q2, bar_kf[P2_NKS], bar_ke[P2_NKS],
-      bar_vf[P2_NVS], bar_ve[P2_NVS], bar_sf[2], bar_pr[2], bar_ph[2], bar_od[2], bar_drain;
+  __shared__ __align__(8) uint64_t bar_q, bar_qg[2], bar_qfree, bar_q2, bar_kf[P2_NKS], bar_kr[P2_NKS],
+      bar_ke[P2_NKS], bar_vf[P2_NVS], bar_ve[P2_NVS], bar_sf[2], bar_pr[2], bar_ph[2], bar_od[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
+  __shared__ KCorrTable kctab;
 
   using GG = Geo<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -724,6 +955,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   const VisitPlan pl = make_plan(t, p.w0);
   const int n_grp = pl.n_grp, n_all = pl.n_all;
   const bool reload_q = n_grp > 0 && n_all > n_grp;
+  const bool kcorr = n_grp > 0 && !p.kg_pre;  // grouped K tiles rotated in this CTA
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
@@ -734,7 +966,11 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     mbar_init(&bar_qg[1], 128);
     mbar_init(&bar_qfree, 1);
     mbar_init(&bar_q2, 1);
-    for (int i = 0; i < P2_NKS; ++i) { mbar_init(&bar_kf[i], 1); mbar_init(&bar_ke[i], 1); }
+    for (int i = 0; i < P2_NKS; ++i) {
+      mbar_init(&bar_kf[i], 1);
+      mbar_init(&bar_kr[i], 128);
+      mbar_init(&bar_ke[i], 1);
+    }
     for (int i = 0; i < P2_NVS; ++i) { mbar_init(&bar_vf[i], 1); mbar_init(&bar_ve[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_sf[i], 1);
@@ -746,12 +982,12 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 9) {
+  if (warp == 13) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_slot)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(&mQ) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&mK) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&mV) : "memory");
@@ -762,9 +998,10 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   const int tok_q0 = a + t.i0;
-  if (warp == 8) {
-    // ================= producer: Q (twice if re-loaded), K tiles in visit order
-    if (lane == 0) {
+  if (warp >= 12) {
+    regs_dec<P2_REG_IO>();
+    if (warp == 12 && lane == 0) {
+      // ================= producer: Q (twice if re-loaded), K tiles in visit order
       mbar_expect_tx(&bar_q, 2 * GG::TB);
       for (int x = 0; x < 2; ++x)
         for (int hf = 0; hf < GG::NH; ++hf)
@@ -787,7 +1024,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         const int st = v % P2_NKS;
         if (v >= P2_NKS && !(ok = wait_b(&bar_ke[st], ((v / P2_NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
           break;
-        const CUtensorMap *m = vv.grp ? &mKg : &mK;
+        const CUtensorMap *m = (vv.grp && p.kg_pre) ? &mKg : &mK;
         const uint32_t dst = sbase + GG::OFF_K + st * GG::TB;
         mbar_expect_tx(&bar_kf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
@@ -798,7 +1035,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         wait_drain(&bar_kf[u % P2_NKS], (u / P2_NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
       wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
       if (q2) wait_drain(&bar_q2, 0, p.err, ERR_TIMEOUT_PRODUCER);
-    } else if (lane == 1) {
+    } else if (warp == 12 && lane == 1) {
       // ================= producer: V tiles in visit order
       bool ok = true;
       int v = 0;
@@ -817,14 +1054,12 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       }
       for (int u = max(0, v - P2_NVS); u < v; ++u)
         wait_drain(&bar_vf[u % P2_NVS], (u / P2_NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
-    }
-  } else if (warp == 9) {
-    // ================= MMA issuer (one thread), fixed order:
-    //   QK_A(0) QK_B(0), then per visit v: PV_A(v) QK_A(v+1) PV_B(v) QK_B(v+1)
-    // so that each softmax warpgroup's next S is computed while the other
-    // head's PV runs.  S_x is reused by QK_x(v+1) only after PV_x(v) (which
-    // read P_x(v) from it) has been issued.
-    if (lane == 0) {
+    } else if (warp == 13 && lane == 0) {
+      // ================= MMA issuer (one thread), fixed order:
+      //   QK_A(0) QK_B(0), then per visit v: PV_A(v) QK_A(v+1) PV_B(v) QK_B(v+1)
+      // so that each softmax warpgroup's next S is computed while the other
+      // head's PV runs.  S_x is reused by QK_x(v+1) only after PV_x(v) (which
+      // read P_x(v) from it) has been issued.
       bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
       if (ok && n_grp > 0)
         ok = wait_b(&bar_qg[0], 0, &abort_flag, p.err, ERR_TIMEOUT_MMA) &&
@@ -838,7 +1073,11 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
           if (!wait_b(&bar_q2, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
           q2_seen = true;
         }
-        if (!wait_b(&bar_kf[v % P2_NKS], (v / P2_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        // a grouped K tile is read once the key correction has rotated it
+        if (x == 0) {
+          uint64_t *kready = (v < n_grp && kcorr) ? &bar_kr[v % P2_NKS] : &bar_kf[v % P2_NKS];
+          if (!wait_b(kready, (v / P2_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        }
         tc_fence_after();
         const uint32_t qaddr = sbase + P2_OFF_Q + x * GG::TB;
         const uint32_t kaddr = sbase + GG::OFF_K + (v % P2_NKS) * GG::TB;
@@ -884,8 +1123,17 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       umma_commit(&bar_drain);
       wait_drain(&bar_drain, 0, p.err, ERR_TIMEOUT_MMA);
     }
+  } else if (warp >= 8) {
+    // ================= key correction (warps 8-11)
+    regs_dec<P2_REG_KCORR>();
+    if (kcorr) {
+      KeyCorrection<D, P2_NKS> kc;
+      kc.init(threadIdx.x - 256, pl.g_begin * BN, t.G, inv, kctab, 1);
+      kc.run(n_grp, sbase + GG::OFF_K, GG::TB, bar_kf, bar_kr, kctab, &abort_flag, p.err);
+    }
   } else {
     // ================= softmax warpgroups (warps 0-3: head A, 4-7: head B)
+    regs_inc<P2_REG_SOFTMAX>();
     const int hx = warp >> 2;
     const int r = threadIdx.x & 127;  // query row within the tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -955,25 +1203,24 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
           if constexpr (MASKED) return (c < cmin || c > cmax) ? -INFINITY : __uint_as_float(raw);
           else return __uint_as_float(raw);
         };
-        // pass 1: row max; the four 32-column loads are in flight together
+        // one pass over TMEM: the four 32-column loads are in flight
+        // together and the row's 128 scores stay in registers
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(scol + 0, r0);
+        tmem_ld32(scol + 32, r1);
+        tmem_ld32(scol + 64, r2);
+        tmem_ld32(scol + 96, r3);
+        tmem_wait_ld_regs(r0);
+        tmem_wait_ld_regs(r1);
+        tmem_wait_ld_regs(r2);
+        tmem_wait_ld_regs(r3);
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        {
-          uint32_t r0[32], r1[32], r2[32], r3[32];
-          tmem_ld32(scol + 0, r0);
-          tmem_ld32(scol + 32, r1);
-          tmem_ld32(scol + 64, r2);
-          tmem_ld32(scol + 96, r3);
-          tmem_wait_ld_regs(r0);
-          tmem_wait_ld_regs(r1);
-          tmem_wait_ld_regs(r2);
-          tmem_wait_ld_regs(r3);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            m4[0] = fmaxf(m4[0], sel(e, r0[e]));
-            m4[1] = fmaxf(m4[1], sel(e + 32, r1[e]));
-            m4[2] = fmaxf(m4[2], sel(e + 64, r2[e]));
-            m4[3] = fmaxf(m4[3], sel(e + 96, r3[e]));
-          }
+        for (int e = 0; e < 32; ++e) {
+          m4[0] = fmaxf(m4[0], sel(e, r0[e]));
+          m4[1] = fmaxf(m4[1], sel(e + 32, r1[e]));
+          m4[2] = fmaxf(m4[2], sel(e + 64, r2[e]));
+          m4[3] = fmaxf(m4[3], sel(e + 96, r3[e]));
         }
         const float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;
         const float m_new = fmaxf(m_run, mt);
@@ -988,54 +1235,43 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
             m_run = m_new;
           }
 #pragma unroll
-          for (int c4 = 0; c4 < D / 32; ++c4) {
-            uint32_t rr[32];
-            tmem_ld32(ocol + c4 * 32, rr);
-            tmem_wait_ld_regs(rr);
+          for (int c4 = 0; c4 < D / 16; ++c4) {
+            uint32_t rr[16];
+            tmem_ld16(ocol + c4 * 16, rr);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
-            tmem_st32(ocol + c4 * 32, rr);
+            for (int e = 0; e < 16; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * f);
+            tmem_st16(ocol + c4 * 16, rr);
           }
           tmem_wait_st();
         }
-        // pass 2: P = exp2(s * scale - m) as bf16 pairs, 64 columns per round
-        // trip; chunk c4's 16 packed columns land on columns 16 c4 .. 16 c4 + 15,
-        // which have already been read
+        // P = exp2(s * scale - m) as bf16 pairs: the 32 columns from c0 land
+        // on TMEM columns c0 / 2 .. c0 / 2 + 15 (already read)
         const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        auto emit = [&](const uint32_t(&rr)[32], int c0) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(scol + h2 * 64, ra);
-          tmem_ld32(scol + h2 * 64 + 32, rb);
-          tmem_wait_ld_regs(ra);
-          tmem_wait_ld_regs(rb);
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t(&rr)[32] = half ? rb : ra;
-            const int c0 = h2 * 64 + half * 32;
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = c0 + 2 * e;
-              const float x0 = sel(c, rr[2 * e]);
-              const float x1 = sel(c + 1, rr[2 * e + 1]);
-              const float2 a2 = ffma2(make_float2(x0, x1), make_float2(p.sl2, p.sl2), make_float2(-m_use, -m_use));
-              const float p0 = ex2(a2.x);
-              const float p1 = ex2(a2.y);
-              if (e & 1) l2b = fadd2(l2b, make_float2(p0, p1));
-              else l2a = fadd2(l2a, make_float2(p0, p1));
-              __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-              pk[e] = *reinterpret_cast<uint32_t *>(&pb);
-            }
-            tmem_st16(scol + (c0 >> 1), pk);
+          for (int e = 0; e < 16; ++e) {
+            const int c = c0 + 2 * e;
+            const float x0 = sel(c, rr[2 * e]);
+            const float x1 = sel(c + 1, rr[2 * e + 1]);
+            const float2 a2 = ffma2(make_float2(x0, x1), make_float2(p.sl2, p.sl2), make_float2(-m_use, -m_use));
+            const float p0 = ex2(a2.x);
+            const float p1 = ex2(a2.y);
+            if (e & 1) l2b = fadd2(l2b, make_float2(p0, p1));
+            else l2a = fadd2(l2a, make_float2(p0, p1));
+            __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+            pk[e] = *reinterpret_cast<uint32_t *>(&pb);
           }
-          if (h2 == 0) {
-            // keys 0-63 of P are in TMEM: the first half of PV may start
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bar_ph[hx]);
-          }
-        }
+          tmem_st16(scol + (c0 >> 1), pk);
+        };
+        emit(r0, 0);
+        emit(r1, 32);
+        // keys 0-63 of P are in TMEM: the first half of PV may start
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar_ph[hx]);
+        emit(r2, 64);
+        emit(r3, 96);
       };
       if (vv.mask)
         visit_body(std::true_type{});
@@ -1082,7 +1318,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
   }
@@ -1123,9 +1359,12 @@ EncodeTiledFn get_encode_tiled() {
   return fn;
 }
 
+// Workspace: a 256-byte error word; with JL_FLAG_PREROTATE_K (the ablation of
+// the in-tile key correction) also the grouped keys K_g, laid out like K.
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags) {
-  (void)batch; (void)Hq; (void)flags;
-  return 256 + a256((size_t)T_total * Hkv * D * 2);
+  (void)batch; (void)Hq;
+  const bool pre = (flags & JL_FLAG_PREROTATE_K) != 0;
+  return 256 + (pre ? a256((size_t)T_total * Hkv * D * 2) : 0);
 }
 
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
@@ -1133,24 +1372,26 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
                               int max_seqlen, int Hq, int Hkv, int D, long long w_pre, int w0, int window,
                               const InvFreq &inv, int plain, uint32_t flags, void *ws, size_t ws_bytes,
                               cudaStream_t st, const char **why) {
-  (void)flags; (void)ws_bytes;
+  (void)ws_bytes;
   const bool pair_heads = ((Hq / Hkv) % 2) == 0;  // two heads of one GQA group per CTA
   if (D != 128 && D != 64) {
     *why = "tensor-core prefill: head_dim 64 or 128";
     return cudaErrorInvalidValue;
   }
   int *err = reinterpret_cast<int *>(ws);
-  __nv_bfloat16 *kg = reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(ws) + 256);
+  // grouped keys are needed unless the window keeps every visible pair local
+  const bool any_grouped = !plain && !(window > 0 && window <= w0);
+  const bool pre = (flags & JL_FLAG_PREROTATE_K) != 0 && any_grouped;
+  __nv_bfloat16 *kg = pre ? reinterpret_cast<__nv_bfloat16 *>(reinterpret_cast<char *>(ws) + 256) : nullptr;
   CUtensorMap mQ, mK, mV, mKg;
   if (!make_map(&mQ, q, T_total, Hq, D) || !make_map(&mK, k, Tk, Hkv, D) || !make_map(&mV, v, Tk, Hkv, D) ||
-      !make_map(&mKg, kg, Tk, Hkv, D)) {
+      !make_map(&mKg, pre ? (const void *)kg : k, Tk, Hkv, D)) {
     *why = "cuTensorMapEncodeTiled failed";
     return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
-  // grouped keys are needed unless the window keeps every visible pair local
-  if (!plain && !(window > 0 && window <= w0)) {
+  if (pre) {
     const long long n = (long long)Tk * (D / 16);
     tc::prerotate_k_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(
         (const __nv_bfloat16 *)k, kg, D, cu_k, batch, Tk, Hkv, w_pre, inv);
@@ -1185,6 +1426,7 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   p.w0 = w0;
   p.plain = plain;
   p.window = window;
+  p.kg_pre = pre ? 1 : 0;
   p.out = (__nv_bfloat16 *)out;
   p.lse = lse;
   p.err = err;
@@ -1200,10 +1442,10 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   } else {
     dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq, batch);
     if (D == 128)
-      tc::bifocal_prefill_kernel<128><<<grid, tc::NUM_THREADS, tc::Geo<128>::P1_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg,
+      tc::bifocal_prefill_kernel<128><<<grid, tc::P1_THREADS, tc::Geo<128>::P1_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg,
                                                                                                   p, inv);
     else
-      tc::bifocal_prefill_kernel<64><<<grid, tc::NUM_THREADS, tc::Geo<64>::P1_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p,
+      tc::bifocal_prefill_kernel<64><<<grid, tc::P1_THREADS, tc::Geo<64>::P1_SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p,
                                                                                                 inv);
   }
   e = cudaGetLastError();
@@ -1243,3 +1485,10 @@ extern "C" int jl_debug_prefill_visits(int L, int Lk, int w0, int window, int G,
   }
   return pl.n_all;
 }
+
+namespace jl {
+// Test hook: the limit of the bounded waits of this file's kernels.
+cudaError_t set_wait_limit_prefill(unsigned long long ns) {
+  return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
+}
+}  // namespace jl

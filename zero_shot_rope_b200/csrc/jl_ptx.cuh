@@ -61,17 +61,32 @@ __device__ __forceinline__ uint64_t gtime() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
+// Bounded waits.  The limit of an ordinary wait is this device variable (one
+// copy per translation unit), 2 s unless a test shortens it through
+// jl_debug_set_wait_limit; the drain waits below keep a fixed 2 s.
+static __device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+
+// A translation unit whose kernels rebalance registers with setmaxnreg
+// defines JL_WAITS_INLINE before including this file: ptxas cannot compile
+// function calls inside such kernels, so the slow paths are inlined there.
+#ifdef JL_WAITS_INLINE
+#define JL_WAIT_SLOW __forceinline__
+#else
+#define JL_WAIT_SLOW __noinline__
+#endif
+
 // Bounded wait: false on timeout (records `code`) or when another role aborted.
 // The first probe is inlined: most waits on the pipelines' critical paths find
 // the phase already complete, and a call there costs more than the probe.
-static __device__ __noinline__ bool wait_b_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                         int *gerr, int code) {
+static __device__ JL_WAIT_SLOW bool wait_b_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                                int *gerr, int code) {
   const uint64_t t0 = gtime();
+  const uint64_t limit = *(volatile unsigned long long *)&g_wait_limit_ns;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
-      if (gtime() - t0 > 2000000000ull) {
+      if (gtime() - t0 > limit) {
         *abort_flag = 1;
         if (gerr) atomicOr(gerr, code);
         return false;
@@ -85,8 +100,8 @@ __device__ __forceinline__ bool wait_b(uint64_t *bar, uint32_t parity, volatile 
   return wait_b_slow(bar, parity, abort_flag, gerr, code);
 }
 // Bounded wait used only to let this CTA's own copies / MMAs land before it
-// exits; ignores the abort flag.
-static __device__ __noinline__ void wait_drain(uint64_t *bar, uint32_t parity, int *gerr, int code) {
+// exits; ignores the abort flag and keeps a fixed limit.
+static __device__ JL_WAIT_SLOW void wait_drain(uint64_t *bar, uint32_t parity, int *gerr, int code) {
   const uint64_t t0 = gtime();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try(bar, parity)) return;

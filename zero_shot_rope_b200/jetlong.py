@@ -20,6 +20,7 @@ JL_OK, JL_ERR_INVALID_ARG, JL_ERR_UNSUPPORTED, JL_ERR_CUDA, JL_ERR_WORKSPACE = r
 JL_BF16, JL_FP32 = 0, 1
 JL_FLAG_PLAIN_CAUSAL = 0x1
 JL_FLAG_SIMT = 0x2
+JL_FLAG_PREROTATE_K = 0x4
 
 _lib = None
 
@@ -72,6 +73,8 @@ def lib() -> ctypes.CDLL:
                                             c_i64, c_i32, c_d, c_p, c_p, ctypes.c_int, c_u32, c_p]
     L.jl_bifocal_decode_noalloc_error.restype = ctypes.c_int
     L.jl_bifocal_decode_noalloc_error.argtypes = [ctypes.POINTER(c_i32), c_p]
+    L.jl_debug_set_wait_limit.restype = ctypes.c_int
+    L.jl_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
     _lib = L
     return L
 
