@@ -39,6 +39,15 @@ def _check_tile(lib, L, Lk, w0, W, G, qt):
         grouped[:, cols] |= keep & bool(grp)
     assert np.array_equal(claims, visible.astype(np.int64)), (L, Lk, w0, W, G, qt)
     assert np.array_equal(grouped[visible], grouped_expected[visible]), (L, Lk, w0, W, G, qt)
+    # the order the kernels rely on: every base visit before every grouped
+    # one (the query tile is rotated in place between the two phases), and
+    # the grouped visits on consecutive key tiles in ascending order (the key
+    # correction advances its rotation by one tile per grouped visit)
+    g = visits[:, 1]
+    if len(g):
+        assert np.all(np.diff(g) >= 0), (L, Lk, w0, W, G, qt)
+        gk = visits[g == 1, 0]
+        assert np.array_equal(gk, np.arange(gk[0], gk[0] + len(gk)) if len(gk) else gk), (L, Lk, w0, W, G, qt)
 
 
 def _lib():

@@ -160,6 +160,16 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float2 f) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 x;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(x.x), "=r"(x.y), "=r"(x.z), "=r"(x.w) : "r"(a));
+  return x;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 x) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x.x), "r"(x.y), "r"(x.z), "r"(x.w)
+               : "memory");
+}
+
 // byte offset of (row, 16-byte chunk) in a 16-row K-major SWIZZLE_128B operand
 // half (rows 128 B apart, chunk XOR-swizzled by row % 8)
 __device__ __forceinline__ int op_off(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
@@ -420,11 +430,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     bool ok = true;
     for (int u = 0; u < ntiles && ok; ++u) {
       const int sk = u % NKS;
+      const int j0 = kb + u * TK;
+      const bool rot_tile = bif && j0 < j_local;
       ok = __all_sync(0xffffffffu, wait_b(&bar_kf[sk], (u / NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT));
       if (!ok) break;
-      const int j0 = kb + u * TK;
-      if (bif && j0 < j_local) {
-        uint8_t *kt = gbase + GG::OFF_K + sk * GG::TB;
+      if (rot_tile) {
+        const uint32_t kt = sbase + GG::OFF_K + sk * GG::TB;
+        // every row's data is read before any row is written back, so the
+        // shared-memory latencies overlap
+        uint4 xa[NR], xb[NR];
+#pragma unroll
+        for (int m = 0; m < NR; ++m) {
+          const int r = r0 + RS * m;
+          xa[m] = lds128(kt + r * 128 + offa);
+          xb[m] = lds128(kt + r * 128 + offb);
+        }
 #pragma unroll
         for (int m = 0; m < NR; ++m) {
           const int r = r0 + RS * m;
@@ -439,10 +459,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
             } else {
               compose(2 * (m - 1) + (rho + smm[m] >= G ? 1 : 0), rc, rs);
             }
-            uint4 *pa = reinterpret_cast<uint4 *>(kt + r * 128 + offa);
-            uint4 *pb = reinterpret_cast<uint4 *>(kt + r * 128 + offb);
-            uint4 xa = *pa, xb = *pb;
-            uint32_t *ua = reinterpret_cast<uint32_t *>(&xa), *ub = reinterpret_cast<uint32_t *>(&xb);
+            uint32_t *ua = reinterpret_cast<uint32_t *>(&xa[m]), *ub = reinterpret_cast<uint32_t *>(&xb[m]);
 #pragma unroll
             for (int e2 = 0; e2 < 4; ++e2) {
               const float2 fa = bf2_to_f2(ua[e2]), fb = bf2_to_f2(ub[e2]);
@@ -451,8 +468,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
               ua[e2] = f2_to_bf2(fma2(fa, cc, mul2(fb, ss)));
               ub[e2] = f2_to_bf2(sub2(mul2(fb, cc), mul2(fa, ss)));
             }
-            *pa = xa;
-            *pb = xb;
+            sts128(kt + r * 128 + offa, xa[m]);
+            sts128(kt + r * 128 + offb, xb[m]);
           }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

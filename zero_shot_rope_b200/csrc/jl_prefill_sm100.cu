@@ -55,7 +55,7 @@ constexpr int P1_THREADS = 384;
 constexpr uint32_t P1_REG_SOFTMAX = 232, P1_REG_IO = 104, P1_REG_KCORR = 168;  // 232 + 104 + 168 = 3 x 168
 // two heads per CTA: softmax A | softmax B | key correction | producers + MMA
 constexpr int P2_THREADS = 512;
-constexpr uint32_t P2_REG_SOFTMAX = 176, P2_REG_KCORR = 88, P2_REG_IO = 72;  // 2 x 176 + 88 + 72 = 4 x 128
+constexpr uint32_t P2_REG_SOFTMAX = 176, P2_REG_KCORR = 96, P2_REG_IO = 64;  // 2 x 176 + 96 + 64 = 4 x 128
 
 // error codes (bit flags) written to the workspace error word
 constexpr int ERR_TIMEOUT_PRODUCER = 1;
@@ -224,10 +224,10 @@ struct Tile {
   int L, G, i0, i1, qt, bif, Lk, off, W;
 };
 
-// Visits of a query tile, in order: the grouped visits (key tiles whose
-// pairs include a distance in [w0, W)) on key tiles g_begin ..
-// g_begin + n_grp - 1, then the base visits (pairs with distance
-// < min(w0, W)) on key tiles ks_begin .. the last key tile.  A visit's
+// Visits of a query tile, in order: the base visits (pairs with distance
+// < min(w0, W)) on key tiles ks_begin .. the last key tile, then the grouped
+// visits (key tiles whose pairs include a distance in [w0, W)) on key tiles
+// g_begin .. g_begin + n_grp - 1, ascending.  A visit's
 // columns c with (p_i - j0 - c) outside [lo, hi] are masked when `mask` is
 // set.  Everything is computed from integers in registers (no per-visit
 // arrays).
@@ -274,8 +274,9 @@ __host__ __device__ __forceinline__ VisitPlan make_plan(const Tile &t, int w0) {
 
 __host__ __device__ __forceinline__ void visit_at(const Tile &t, const VisitPlan &pl, int w0, int v, int &kt,
                                                   Visit &out) {
-  const bool grp = v < pl.n_grp;
-  kt = grp ? pl.g_begin + v : pl.ks_begin + (v - pl.n_grp);
+  const int n_base = pl.n_all - pl.n_grp;
+  const bool grp = v >= n_base;
+  kt = grp ? pl.g_begin + (v - n_base) : pl.ks_begin + v;
   const int j0 = kt * BN;
   const int j1 = min(j0 + BN - 1, t.Lk - 1);
   const int dmin = t.off + t.i0 - j1, dmax = t.off + t.i1 - j0;
@@ -399,13 +400,22 @@ struct KeyCorrection {
       s[w] = bs[w];
     }
     int rr = rho;  // key index of the current row, mod G
+    auto addr_a = [&](int row) { return tile + row * 128 + ((lc ^ (row & 7)) << 4); };
+    auto addr_b = [&](int row) {
+      return D == 128 ? tile + HALF_BYTES + row * 128 + ((lc ^ (row & 7)) << 4)
+                      : tile + row * 128 + (((lc + 4) ^ (row & 7)) << 4);
+    };
+    // row m + 1 is read before row m is written back, so each row's
+    // shared-memory latency overlaps the previous row's arithmetic
+    uint4 na = lds128(addr_a(r0)), nb = lds128(addr_b(r0));
 #pragma unroll 1
     for (int m = 0; m < RPT; ++m) {
       const int row = r0 + m;
-      const int sw = row & 7;
-      const uint32_t pa = tile + row * 128 + ((lc ^ sw) << 4);
-      const uint32_t pb = D == 128 ? pa + HALF_BYTES : tile + row * 128 + (((lc + 4) ^ sw) << 4);
-      uint4 xa = lds128(pa), xb = lds128(pb);
+      uint4 xa = na, xb = nb;
+      if (m + 1 < RPT) {
+        na = lds128(addr_a(row + 1));
+        nb = lds128(addr_b(row + 1));
+      }
       uint32_t *ua = reinterpret_cast<uint32_t *>(&xa), *ub = reinterpret_cast<uint32_t *>(&xb);
       // R(-n) (a, b) = (a cos + b sin, b cos - a sin)
 #pragma unroll
@@ -414,8 +424,8 @@ struct KeyCorrection {
         ua[w] = f2_bf2(__ffma2_rn(fa, c[w], __fmul2_rn(fb, s[w])));
         ub[w] = f2_bf2(__ffma2_rn(fb, c[w], __fmul2_rn(neg2(fa), s[w])));
       }
-      sts128(pa, xa);
-      sts128(pb, xb);
+      sts128(addr_a(row), xa);
+      sts128(addr_b(row), xb);
       if (m + 1 < RPT) {
         if (rr + 1 == G) {
           rr = 0;  // the next key starts a group: n unchanged
@@ -442,19 +452,21 @@ struct KeyCorrection {
     rho += sigma - (carry ? G : 0);
   }
 
-  // The role: for the grouped visits v = 0 .. n_grp - 1 (key tiles in
-  // ascending order, the first visits of the CTA), wait for the K tile of
-  // stage v % NSTAGE, rotate it, make the writes visible to the tensor core
-  // and release it to the MMA issuer.
-  __device__ __forceinline__ void run(int n_grp, uint32_t kring, int stage_bytes, uint64_t *bar_kf,
+  // The role: every visit's K tile passes through here (stage v % NSTAGE,
+  // in visit order); the grouped visits' tiles, the last n_grp visits on key
+  // tiles in ascending order, are rotated, and each tile is then made visible
+  // to the tensor core and released to the MMA issuer.
+  __device__ __forceinline__ void run(int n_all, int n_grp, uint32_t kring, int stage_bytes, uint64_t *bar_kf,
                                       uint64_t *bar_kr, const KCorrTable &tab, volatile int *abort_flag,
                                       int *err) {
-    for (int v = 0; v < n_grp; ++v) {
+    for (int v = 0; v < n_all; ++v) {
       const int st = v % NSTAGE;
       if (!__all_sync(0xffffffffu, wait_b(&bar_kf[st], (v / NSTAGE) & 1, abort_flag, err, ERR_TIMEOUT_KCORR)))
         break;
-      rotate_tile(kring + st * stage_bytes, tab);
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (v >= n_all - n_grp) {
+        rotate_tile(kring + st * stage_bytes, tab);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
       mbar_arrive(&bar_kr[st]);
     }
   }
@@ -556,7 +568,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     if (kcorr) {
       KeyCorrection<D, P1_NKS> kc;
       kc.init(threadIdx.x - 256, pl.g_begin * BN, t.G, inv, kctab, 1);
-      kc.run(pl.n_grp, sbase + OFF_K1, GG::TB, bar_kf, bar_kr, kctab, &abort_flag, p.err);
+      kc.run(pl.n_all, pl.n_grp, sbase + OFF_K1, GG::TB, bar_kf, bar_kr, kctab, &abort_flag, p.err);
     }
   } else if (warp >= 4) {
     regs_dec<P1_REG_IO>();
@@ -628,8 +640,9 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
           qg_seen = true;
         }
         const int st = v % P1_NKS;
-        // a grouped K tile is read once the key correction has rotated it
-        uint64_t *kready = (vx.grp && kcorr) ? &bar_kr[st] : &bar_kf[st];
+        // with the key correction running, every K tile passes through it
+        // (the grouped ones rotated) before the MMA reads it
+        uint64_t *kready = kcorr ? &bar_kr[st] : &bar_kf[st];
         if (!(ok = wait_b(kready, (v / P1_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
         tc_fence_after();
         const uint32_t qaddr = sbase + (vx.grp ? GG::P1_OFF_QG : OFF_Q);
@@ -923,7 +936,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
                         const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mKg,
                         const __grid_constant__ Params p, const __grid_constant__ InvFreq inv) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_qg[2], bar_qfree, bar_q2, bar_kf[P2_NKS], bar_kr[P2_NKS],
+  __shared__ __align__(8) uint64_t bar_q, bar_qg[2], bar_kf[P2_NKS], bar_kr[P2_NKS],
       bar_ke[P2_NKS], bar_vf[P2_NVS], bar_ve[P2_NVS], bar_sf[2], bar_pr[2], bar_ph[2], bar_od[2], bar_drain;
   __shared__ uint32_t tmem_slot;
   __shared__ volatile int abort_flag;
@@ -954,7 +967,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   // visits: grouped ones first
   const VisitPlan pl = make_plan(t, p.w0);
   const int n_grp = pl.n_grp, n_all = pl.n_all;
-  const bool reload_q = n_grp > 0 && n_all > n_grp;
+  const int n_base = n_all - n_grp;            // base visits first, then grouped
   const bool kcorr = n_grp > 0 && !p.kg_pre;  // grouped K tiles rotated in this CTA
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
@@ -964,8 +977,6 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     mbar_init(&bar_q, 1);
     mbar_init(&bar_qg[0], 128);
     mbar_init(&bar_qg[1], 128);
-    mbar_init(&bar_qfree, 1);
-    mbar_init(&bar_q2, 1);
     for (int i = 0; i < P2_NKS; ++i) {
       mbar_init(&bar_kf[i], 1);
       mbar_init(&bar_kr[i], 128);
@@ -1001,26 +1012,17 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   if (warp >= 12) {
     regs_dec<P2_REG_IO>();
     if (warp == 12 && lane == 0) {
-      // ================= producer: Q (twice if re-loaded), K tiles in visit order
+      // ================= producer: Q, then K tiles in visit order
       mbar_expect_tx(&bar_q, 2 * GG::TB);
       for (int x = 0; x < 2; ++x)
         for (int hf = 0; hf < GG::NH; ++hf)
           tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * GG::TB + hf * HALF_BYTES, 64 * hf, hA + x, tok_q0);
-      bool ok = true, q2 = false;
+      bool ok = true;
       int v = 0;
       for (; ok && v < n_all;) {
         int kt;
         Visit vv;
         visit_at(t, pl, p.w0, v, kt, vv);
-        if (!vv.grp && reload_q && !q2) {
-          // base phase: the grouped QKs are done with the rotated tiles
-          if (!(ok = wait_b(&bar_qfree, 0, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER))) break;
-          mbar_expect_tx(&bar_q2, 2 * GG::TB);
-          for (int x = 0; x < 2; ++x)
-            for (int hf = 0; hf < GG::NH; ++hf)
-              tma_load(&mQ, &bar_q2, sbase + P2_OFF_Q + x * GG::TB + hf * HALF_BYTES, 64 * hf, hA + x, tok_q0);
-          q2 = true;
-        }
         const int st = v % P2_NKS;
         if (v >= P2_NKS && !(ok = wait_b(&bar_ke[st], ((v / P2_NKS) - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_PRODUCER)))
           break;
@@ -1034,7 +1036,6 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       for (int u = max(0, v - P2_NKS); u < v; ++u)
         wait_drain(&bar_kf[u % P2_NKS], (u / P2_NKS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
       wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
-      if (q2) wait_drain(&bar_q2, 0, p.err, ERR_TIMEOUT_PRODUCER);
     } else if (warp == 12 && lane == 1) {
       // ================= producer: V tiles in visit order
       bool ok = true;
@@ -1061,21 +1062,14 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       // head's PV runs.  S_x is reused by QK_x(v+1) only after PV_x(v) (which
       // read P_x(v) from it) has been issued.
       bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
-      if (ok && n_grp > 0)
-        ok = wait_b(&bar_qg[0], 0, &abort_flag, p.err, ERR_TIMEOUT_MMA) &&
-             wait_b(&bar_qg[1], 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
-      bool q2_seen = !reload_q;
       auto issue_qk = [&](int x, int v) -> bool {
-        if (v >= n_grp && !q2_seen) {
-          // first base-phase QK: release the rotated query tiles, wait for
-          // the re-loaded ones
-          umma_commit(&bar_qfree);
-          if (!wait_b(&bar_q2, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
-          q2_seen = true;
-        }
+        // the first grouped QK of a head reads its query tile rotated in
+        // place by that head's softmax warpgroup
+        if (v == n_base && n_grp > 0 && !wait_b(&bar_qg[x], 0, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         // a grouped K tile is read once the key correction has rotated it
+        // (with the key correction running, every K tile passes through it)
         if (x == 0) {
-          uint64_t *kready = (v < n_grp && kcorr) ? &bar_kr[v % P2_NKS] : &bar_kf[v % P2_NKS];
+          uint64_t *kready = kcorr ? &bar_kr[v % P2_NKS] : &bar_kf[v % P2_NKS];
           if (!wait_b(kready, (v / P2_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         }
         tc_fence_after();
@@ -1129,7 +1123,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     if (kcorr) {
       KeyCorrection<D, P2_NKS> kc;
       kc.init(threadIdx.x - 256, pl.g_begin * BN, t.G, inv, kctab, 1);
-      kc.run(n_grp, sbase + GG::OFF_K, GG::TB, bar_kf, bar_kr, kctab, &abort_flag, p.err);
+      kc.run(n_all, n_grp, sbase + GG::OFF_K, GG::TB, bar_kf, bar_kr, kctab, &abort_flag, p.err);
     }
   } else {
     // ================= softmax warpgroups (warps 0-3: head A, 4-7: head B)
@@ -1142,44 +1136,47 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
     const int i = t.i0 + r;
     const int h = hA + hx;
     bool ok = true;
-    if (n_grp > 0) {
-      // rotate this head's query tile in place: Q_g = R(f(i) - i) Q~
-      ok = __all_sync(0xffffffffu, wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
-      if (ok) {
-        uint8_t *qt = gbase + P2_OFF_Q + hx * GG::TB;
-        // pair k = (element k, element k + D/2).  D = 128: chunk u of box 0
-        // pairs with the same chunk of box 1.  D = 64: in the one 128-byte
-        // row, logical chunk lc (elements 8 lc ..) pairs with chunk lc + 4.
-        for (int kk = 0; kk < (D == 128 ? 8 : 4); ++kk) {
-          const int u = r + 128 * kk;
-          const int row = D == 128 ? u >> 3 : u >> 2;
-          const int lc = D == 128 ? (u & 7) ^ (row & 7) : u & 3;
-          const int n = corr_n(t.off + min(t.i0 + row, L - 1), t.G);
-          uint4 *qa = reinterpret_cast<uint4 *>(D == 128 ? qt + u * 16 : qt + row * 128 + ((lc ^ (row & 7)) << 4));
-          uint4 *qb = reinterpret_cast<uint4 *>(D == 128 ? qt + HALF_BYTES + u * 16
-                                                         : qt + row * 128 + (((lc + 4) ^ (row & 7)) << 4));
-          uint4 xa = *qa, xb = *qb;
-          uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
+    // rotate this head's query tile in place, Q_g = R(f(i) - i) Q~, once its
+    // base-phase QK products are done (the S of its last base visit is ready)
+    // or, with no base visit, once it has landed
+    auto rotate_q = [&]() {
+      uint8_t *qt = gbase + P2_OFF_Q + hx * GG::TB;
+      // pair k = (element k, element k + D/2).  D = 128: chunk u of box 0
+      // pairs with the same chunk of box 1.  D = 64: in the one 128-byte
+      // row, logical chunk lc (elements 8 lc ..) pairs with chunk lc + 4.
+      for (int kk = 0; kk < (D == 128 ? 8 : 4); ++kk) {
+        const int u = r + 128 * kk;
+        const int row = D == 128 ? u >> 3 : u >> 2;
+        const int lc = D == 128 ? (u & 7) ^ (row & 7) : u & 3;
+        const int n = corr_n(t.off + min(t.i0 + row, L - 1), t.G);
+        uint4 *qa = reinterpret_cast<uint4 *>(D == 128 ? qt + u * 16 : qt + row * 128 + ((lc ^ (row & 7)) << 4));
+        uint4 *qb = reinterpret_cast<uint4 *>(D == 128 ? qt + HALF_BYTES + u * 16
+                                                       : qt + row * 128 + (((lc + 4) ^ (row & 7)) << 4));
+        uint4 xa = *qa, xb = *qb;
+        uint32_t *pa = reinterpret_cast<uint32_t *>(&xa), *pb = reinterpret_cast<uint32_t *>(&xb);
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pa[e2]));
-            float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pb[e2]));
-            float c0, s0, c1, s1;
-            angle_cs(n, inv.v[lc * 8 + 2 * e2], c0, s0);
-            angle_cs(n, inv.v[lc * 8 + 2 * e2 + 1], c1, s1);
-            rot_back(fa.x, fb.x, c0, s0);
-            rot_back(fa.y, fb.y, c1, s1);
-            __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
-            __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
-            pa[e2] = *reinterpret_cast<uint32_t *>(&ra);
-            pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
-          }
-          *qa = xa;
-          *qb = xb;
+        for (int e2 = 0; e2 < 4; ++e2) {
+          float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pa[e2]));
+          float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&pb[e2]));
+          float c0, s0, c1, s1;
+          angle_cs(n, inv.v[lc * 8 + 2 * e2], c0, s0);
+          angle_cs(n, inv.v[lc * 8 + 2 * e2 + 1], c1, s1);
+          rot_back(fa.x, fb.x, c0, s0);
+          rot_back(fa.y, fb.y, c1, s1);
+          __nv_bfloat162 ra = __floats2bfloat162_rn(fa.x, fa.y);
+          __nv_bfloat162 rb = __floats2bfloat162_rn(fb.x, fb.y);
+          pa[e2] = *reinterpret_cast<uint32_t *>(&ra);
+          pb[e2] = *reinterpret_cast<uint32_t *>(&rb);
         }
+        *qa = xa;
+        *qb = xb;
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(&bar_qg[hx]);
+    };
+    if (n_grp > 0 && n_base == 0) {
+      ok = __all_sync(0xffffffffu, wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+      rotate_q();
     }
 
     float m_run = -INFINITY, l_run = 0.f;
@@ -1189,8 +1186,10 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       Visit vv;
       visit_at(t, pl, p.w0, v, kt, vv);
       ok = __all_sync(0xffffffffu, wait_b(&bar_sf[hx], v & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
-      if (!ok) break;
       tc_fence_after();
+      // the head's last base visit: its QK products (which read Q~) are done
+      if (v == n_base - 1 && n_grp > 0) rotate_q();
+      if (!ok) break;
       // columns c with distance dc - c outside [lo, hi] are masked; the
       // visit-uniform mask flag selects a specialisation without compares
       const int dc = t.off + i - kt * BN;  // row position minus the tile's first key
