@@ -574,8 +574,11 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
     regs_dec<P1_REG_IO>();
     if (warp == 4 && lane == 0) {
       // ================= producer: Q, then K tiles in visit order =================
+      // (K and V are kept in L2 ahead of the query tile, read once)
+      const uint64_t pol_kv = l2_evict_last(), pol_q = l2_evict_first();
       mbar_expect_tx(&bar_q, GG::TB);
-      for (int hf = 0; hf < GG::NH; ++hf) tma_load(&mQ, &bar_q, sbase + OFF_Q + hf * HALF_BYTES, 64 * hf, h, tok_q0);
+      for (int hf = 0; hf < GG::NH; ++hf)
+        tma_load_hint(&mQ, &bar_q, sbase + OFF_Q + hf * HALF_BYTES, 64 * hf, h, tok_q0, pol_q);
       int v = 0;
       for (; v < pl.n_all; ++v) {
         int kt;
@@ -589,7 +592,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         const uint32_t dst = sbase + OFF_K1 + st * GG::TB;
         mbar_expect_tx(&bar_kf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
-          tma_load(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
+          tma_load_hint(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN, pol_kv);
       }
       // drain: every load issued must land before the CTA may exit
       for (int u = max(0, v - P1_NKS); u < v; ++u)
@@ -597,6 +600,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
     } else if (warp == 6 && lane == 0) {
       // ================= producer: V tiles in visit order =================
+      const uint64_t pol_kv = l2_evict_last();
       int v = 0;
       for (; v < pl.n_all; ++v) {
         int kt;
@@ -608,7 +612,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         const uint32_t dst = sbase + OFF_V1 + st * GG::TB;
         mbar_expect_tx(&bar_vf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
-          tma_load(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
+          tma_load_hint(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN, pol_kv);
       }
       for (int u = max(0, v - NVS); u < v; ++u) wait_drain(&bar_vf[u % NVS], (u / NVS) & 1, p.err, ERR_TIMEOUT_PRODUCER);
     } else if (warp == 5 && lane == 0) {
@@ -1012,11 +1016,15 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   if (warp >= 12) {
     regs_dec<P2_REG_IO>();
     if (warp == 12 && lane == 0) {
-      // ================= producer: Q, then K tiles in visit order
+      // ================= producer: Q, then K tiles in visit order.  K and V
+      // tiles are read by every CTA of the kv head: kept in L2 ahead of the
+      // query tiles, which one CTA reads once.
+      const uint64_t pol_kv = l2_evict_last(), pol_q = l2_evict_first();
       mbar_expect_tx(&bar_q, 2 * GG::TB);
       for (int x = 0; x < 2; ++x)
         for (int hf = 0; hf < GG::NH; ++hf)
-          tma_load(&mQ, &bar_q, sbase + P2_OFF_Q + x * GG::TB + hf * HALF_BYTES, 64 * hf, hA + x, tok_q0);
+          tma_load_hint(&mQ, &bar_q, sbase + P2_OFF_Q + x * GG::TB + hf * HALF_BYTES, 64 * hf, hA + x, tok_q0,
+                        pol_q);
       bool ok = true;
       int v = 0;
       for (; ok && v < n_all;) {
@@ -1030,7 +1038,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         const uint32_t dst = sbase + GG::OFF_K + st * GG::TB;
         mbar_expect_tx(&bar_kf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
-          tma_load(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
+          tma_load_hint(m, &bar_kf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN, pol_kv);
         ++v;
       }
       for (int u = max(0, v - P2_NKS); u < v; ++u)
@@ -1038,6 +1046,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       wait_drain(&bar_q, 0, p.err, ERR_TIMEOUT_PRODUCER);
     } else if (warp == 12 && lane == 1) {
       // ================= producer: V tiles in visit order
+      const uint64_t pol_kv = l2_evict_last();
       bool ok = true;
       int v = 0;
       for (; ok && v < n_all;) {
@@ -1050,7 +1059,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         const uint32_t dst = sbase + GG::OFF_V + st * GG::TB;
         mbar_expect_tx(&bar_vf[st], GG::TB);
         for (int hf = 0; hf < GG::NH; ++hf)
-          tma_load(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN);
+          tma_load_hint(&mV, &bar_vf[st], dst + hf * HALF_BYTES, 64 * hf, kvh, ak + kt * BN, pol_kv);
         ++v;
       }
       for (int u = max(0, v - P2_NVS); u < v; ++u)

@@ -120,6 +120,27 @@ __device__ __forceinline__ void tma_load(const CUtensorMap *map, uint64_t *bar, 
       : "memory");
 }
 
+// The same load with an L2 eviction-priority policy (from createpolicy).
+__device__ __forceinline__ void tma_load_hint(const CUtensorMap *map, uint64_t *bar, uint32_t dst, int c0, int c1,
+                                              int c2, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(map), "r"(su32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+      : "memory");
+}
+// L2 policies: keep lines that other CTAs will read again; let once-read lines go first.
+__device__ __forceinline__ uint64_t l2_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ float ex2(float x) {  // MUFU exp2 (ex2.approx.ftz)
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
