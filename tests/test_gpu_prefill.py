@@ -129,6 +129,25 @@ def test_full_size_workload_sampled_rows(name):
         assert diff > 5 * err.mean(), (diff, err.mean())
 
 
+@pytest.mark.parametrize("w_pre,G", [(7000, 3), (3000, 7)])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (3, 1)])
+def test_key_correction_over_many_tiles_with_carries(w_pre, G, Hq, Hkv):
+    # 128 is not a multiple of G = 3 or 7, so the key correction's per-tile
+    # step takes both of its values; over ~150 grouped key tiles the carried
+    # fp32 rotation must stay on the oracle (both kernels; sampled rows,
+    # every head)
+    L, w0 = 20000, 512
+    assert oracle.group_size(L, w_pre) == G
+    q, k, v, cu = synth.random_case(100 + G, (L,), Hq, Hkv, 128, torch.bfloat16)
+    out, lse = prefill_gpu(q, k, v, cu, w_pre, w0, 1e6)
+    rows = sample_rows([L], w0, [G], n_edge=64, n_random=128, seed=G)
+    ro, rl = oracle_rows_threaded(oracle.bifocal_attention, rows, q, k, v, cu, w_pre, w0, 1e6)
+    got = to_np(out)[rows]
+    assert_close(got, ro, torch.bfloat16, "out")
+    assert_close(to_np(lse)[:, rows], rl, torch.bfloat16, "lse")
+    assert np.linalg.norm(got - ro) / np.linalg.norm(ro) < 1e-2
+
+
 def test_planted_needles_peaked_attention():
     # A key planted so that its score with one query is large under the
     # method's own geometry (aligned with the query after the correction

@@ -52,11 +52,13 @@ KV_CASES = [
 
 
 @pytest.mark.parametrize("lq,lk,Hq,Hkv,w_pre,w0", KV_CASES)
-@pytest.mark.parametrize("kernel", ["tensor", "simt"])
+@pytest.mark.parametrize("kernel", ["tensor", "prerotated", "simt"])
 def test_chunk_against_cache_full(lq, lk, Hq, Hkv, w_pre, w0, kernel):
+    # "tensor": grouped keys rotated in the tile; "prerotated": the ablation
+    # that writes them for the whole key set in a pre-pass
     J = jl()
     q, k, v, cu_q, cu_k = chunk_case(sum(lk) + Hq + w0, lq, lk, Hq, Hkv)
-    flags = J.JL_FLAG_SIMT if kernel == "simt" else 0
+    flags = {"tensor": 0, "prerotated": J.JL_FLAG_PREROTATE_K, "simt": J.JL_FLAG_SIMT}[kernel]
     out, lse = prefill_kv_gpu(q, k, v, cu_q, cu_k, w_pre, w0, 1e6, flags=flags)
     ro, rl = oracle.bifocal_attention_kv(q, k, v, cu_q, cu_k, w_pre, w0, 1e6)
     assert_close(to_np(out), ro, torch.bfloat16, "out")

@@ -812,6 +812,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool row_ok = i < L;
+      const uint64_t pol_o = l2_evict_first();  // written once, never read here
       __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -829,7 +830,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
                                                         __uint_as_float(rr[e8 * 8 + 2 * e2 + 1]) * inv_l);
               po[e2] = *reinterpret_cast<uint32_t *>(&ob);
             }
-            *reinterpret_cast<uint4 *>(orow + c4 * 32 + e8 * 8) = o4;
+            stg128_hint(orow + c4 * 32 + e8 * 8, o4, pol_o);
           }
         }
       }
@@ -949,17 +950,22 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
   using GG = Geo<D>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.z;
-  const int hA = 2 * blockIdx.y;  // heads hA, hA + 1 (same kv head: the group size is even)
+  // x enumerates (query tile, head pair of the kv head) with the head pair
+  // fastest, so the CTAs of all head pairs of one kv head run side by side
+  // and sweep the same K and V tiles at the same time (shared in L2)
+  const int ppk = p.Hq / p.Hkv / 2;          // head pairs per kv head
+  const int qx = (int)blockIdx.x / ppk;      // query-tile index (heaviest first)
+  const int hA = 2 * ((int)blockIdx.y * ppk + (int)blockIdx.x % ppk);  // heads hA, hA + 1
   const int a = p.cu[s];                // first query token
   const int L = p.cu[s + 1] - a;        // queries
   const int ak = p.cu_k[s];             // first key token
   const int Lk = p.cu_k[s + 1] - ak;    // keys: the sequence's current length
   if (L <= 0 || a < 0 || a + L > p.T || Lk < L || ak < 0 || ak + Lk > p.Tk) return;
   const int nqt = (L + BM - 1) / BM;
-  if ((int)blockIdx.x >= nqt) return;
+  if (qx >= nqt) return;
   Tile t;
   t.L = L;
-  t.qt = nqt - 1 - (int)blockIdx.x;
+  t.qt = nqt - 1 - qx;
   t.i0 = t.qt * BM;
   t.i1 = min(t.i0 + BM - 1, L - 1);
   t.Lk = Lk;
@@ -1297,6 +1303,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool row_ok = i < L;
+      const uint64_t pol_o = l2_evict_first();  // written once, never read here
       __nv_bfloat16 *orow = p.out + ((size_t)(tok_q0 + r) * p.Hq + h) * D;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -1314,7 +1321,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
                                                         __uint_as_float(rr[e8 * 8 + 2 * e2 + 1]) * inv_l);
               po[e2] = *reinterpret_cast<uint32_t *>(&ob);
             }
-            *reinterpret_cast<uint4 *>(orow + c4 * 32 + e8 * 8) = o4;
+            stg128_hint(orow + c4 * 32 + e8 * 8, o4, pol_o);
           }
         }
       }
@@ -1440,7 +1447,7 @@ cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void 
   p.err = err;
   p.sl2 = 1.4426950408889634f / sqrtf((float)D);
   if (pair_heads) {
-    dim3 grid((max_seqlen + tc::BM - 1) / tc::BM, Hq / 2, batch);
+    dim3 grid((max_seqlen + tc::BM - 1) / tc::BM * (Hq / Hkv / 2), Hkv, batch);
     if (D == 128)
       tc::bifocal_prefill2_kernel<128><<<grid, tc::P2_THREADS, tc::Geo<128>::SMEM_ALLOC, st>>>(mQ, mK, mV, mKg, p,
                                                                                                  inv);

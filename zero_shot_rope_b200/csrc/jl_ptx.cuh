@@ -141,6 +141,13 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   return pol;
 }
 
+// 16-byte global store with an L2 eviction-priority policy.
+__device__ __forceinline__ void stg128_hint(void *p, uint4 x, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(x.x), "r"(x.y), "r"(x.z),
+               "r"(x.w), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ float ex2(float x) {  // MUFU exp2 (ex2.approx.ftz)
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
