@@ -43,6 +43,8 @@ def test_every_attended_key_falls_in_one_split(bf16):
         assert ns * ch >= keys, (B, Hq, Hkv, D, M, W, ns, ch)     # no attended key left out
         assert (ns - 1) * ch < keys, (B, Hq, Hkv, D, M, W, ns, ch)  # no split past the keys
         assert ch % 64 == 0                                        # whole key tiles
+        if bf16 and Hq // Hkv <= 8:  # the tensor-core decode: 256-key tiles at head_dim 64, 128 at 128
+            assert ch % (256 if D == 64 else 128) == 0, (D, ch)
         assert rows >= B * Hq * ns, (B, Hq, Hkv, D, M, W, ns, rows)  # the workspace holds them
 
 

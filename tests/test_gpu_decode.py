@@ -33,6 +33,11 @@ SMALL = [
     ((5000,), 5000, 8, 8, 128, 900, 0, torch.bfloat16),
     ((600,), 700, 8, 1, 128, 100, 600, torch.bfloat16),          # all keys local
     ((700,), 700, 4, 2, 64, 150, 50, torch.bfloat16),
+    # head_dim 64 runs 256-key tiles: one key past a tile, several splits of
+    # ragged lengths with eight query heads per kv head, a single key
+    ((257,), 300, 8, 8, 64, 100, 20, torch.bfloat16),
+    ((3333, 17, 2048), 4000, 16, 2, 64, 700, 300, torch.bfloat16),
+    ((1,), 8, 4, 1, 64, 1, 0, torch.bfloat16),
     ((900, 33), 1000, 4, 4, 64, 200, 10, torch.float32),
     ((2500,), 2600, 16, 2, 128, 512, 100, torch.float32),
 ]

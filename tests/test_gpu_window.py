@@ -94,6 +94,7 @@ DEC = [
     ((1200,), 1200, 8, 8, 128, 300, 0, 5000, torch.bfloat16),        # window > L
     ((900, 33), 1000, 4, 4, 64, 200, 10, 129, torch.float32),        # CUDA-core decode kernel
     ((700,), 700, 4, 2, 64, 150, 50, 333, torch.bfloat16),
+    ((5000, 611), 5000, 16, 4, 64, 900, 100, 700, torch.bfloat16),   # 256-key tiles, window off the grid
 ]
 
 

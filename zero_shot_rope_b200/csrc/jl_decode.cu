@@ -462,7 +462,7 @@ static cudaError_t launch_decode_d(int GS, const CUtensorMap &mK, const CUtensor
   return cudaErrorInvalidValue;
 }
 
-void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk);
+void decode_tc_plan(int batch, int Hkv, int D, int max_seqlen, int *nsplit, int *chunk);
 cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
                              const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
                              int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
@@ -485,12 +485,13 @@ size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
 }
 
 static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv, int D) {
-  // bf16 cache viewed as (d, head, row); 64 x 1 x 128 boxes, 128-byte swizzle
+  // bf16 cache viewed as (d, head, row); 64 x 1 x (keys of a tile) boxes,
+  // 128-byte swizzle: 128 keys at head_dim 128, 256 at 64
   EncodeTiledFn enc = get_encode_tiled();
   if (enc == nullptr) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
-  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t box[3] = {64, 1, D == 64 ? 256u : 128u};
   cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -509,7 +510,7 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
     if (!make_tile_map(&tK, kc, B * Lcap, Hkv, D) || !make_tile_map(&tV, vc, B * Lcap, Hkv, D))
       return cudaErrorInvalidValue;
     int ns, chunk;
-    decode_tc_plan(B, Hkv, keys, &ns, &chunk);
+    decode_tc_plan(B, Hkv, D, keys, &ns, &chunk);
     cudaError_t e = launch_decode_tc(GS, D, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, Hq, Hkv, w_pre, w0,
                                      window, inv, plain, ns, chunk, part_o, part_ml, err, st);
     if (e != cudaSuccess) return e;
@@ -701,7 +702,7 @@ extern "C" int jl_debug_decode_plan(int batch, int Hq, int Hkv, int D, int max_s
   const int GS = Hq / Hkv;
   const int keys = window > 0 ? min(max_seqlen, window) : max_seqlen;
   if (jl::use_tc_decode(bf16 != 0, D, GS)) {
-    jl::decode_tc_plan(batch, Hkv, keys, nsplit, chunk);
+    jl::decode_tc_plan(batch, Hkv, D, keys, nsplit, chunk);
   } else {
     const jl::DecodePlan pl = jl::decode_plan(batch, Hq, Hkv, D, keys, bf16 ? 2 : 4);
     *nsplit = pl.nsplit;

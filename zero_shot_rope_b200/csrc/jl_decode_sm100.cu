@@ -36,7 +36,11 @@
 namespace jl {
 namespace dtc {
 
-constexpr int TK = 128;   // keys per tile
+// keys per tile: 128 at head_dim 128; 256 at head_dim 64, so that a K or V
+// stage holds 32 KB and a tile's fixed costs (products, softmax exchange,
+// barriers) are spread over as many bytes as at head_dim 128
+template <int D>
+constexpr int tile_keys() { return D == 64 ? 256 : 128; }
 constexpr int NROT = 8;                          // rotation warps
 constexpr int THREADS = 128 + NROT * 32 + 64;   // softmax + rotation + TMA + MMA
 constexpr int WARP_TMA = 4 + NROT;
@@ -44,8 +48,7 @@ constexpr int WARP_MMA = 5 + NROT;
 
 constexpr int NKS = 3;    // K ring stages
 constexpr int NVS = 3;    // V ring stages
-constexpr int HALF_BYTES = TK * 64 * 2;  // one 64-column SWIZZLE_128B box of a 128-row tile
-constexpr int POPB = 16 * 128 * 2;       // the P operand: 16 rows x 128 keys (2 boxes)
+constexpr int HALF_BYTES = 128 * 64 * 2;  // one 64-column SWIZZLE_128B box of a 128-row tile (D = 128)
 
 // Geometry for a head_dim D (64 or 128).  A K or V tile row is D / 64 boxes;
 // the Q operand is 16 rows x D.  PV is O^T = V^T P with M = 128: at D = 64 the
@@ -53,8 +56,11 @@ constexpr int POPB = 16 * 128 * 2;       // the P operand: 16 rows x 128 keys (2
 // so O^T rows 64-127 stay zero and the TMEM layout is that of D = 128.
 template <int D>
 struct Geo {
+  static constexpr int TK = tile_keys<D>();
   static constexpr int NH = D / 64;
-  static constexpr int TB = TK * D * 2;
+  static constexpr int TB = TK * D * 2;             // one K or V tile: 32 KB
+  static constexpr int PBOX = 16 * 64 * 2;          // one 64-key box of the P operand
+  static constexpr int POPB = PBOX * (TK / 64);     // the P operand: 16 rows x TK keys
   static constexpr int QOPB = 16 * D * 2;
   static constexpr int KSTEPS = D / 16;            // k-steps of S^T = K Q^T
   static constexpr int OFF_K = 0;
@@ -62,6 +68,11 @@ struct Geo {
   static constexpr int OFF_Q = OFF_V + NVS * TB;
   static constexpr int OFF_P = OFF_Q + (QOPB < 1024 ? 1024 : QOPB);
   static constexpr int OFF_Z = OFF_P + 2 * POPB;   // zero block (D = 64)
+  // TMEM: S^T of the two tiles in flight, TK / 128 blocks of 16 columns
+  // each, then O^T
+  static constexpr uint32_t S_COLS = 16 * (TK / 128);
+  static constexpr uint32_t COL_O = 2 * S_COLS;
+  static constexpr uint32_t TMEM_COLS = COL_O + 16 <= 64 ? 64 : 128;
   static constexpr int SMEM_ALLOC = OFF_Z + (D == 64 ? 2048 : 0) + 1024;
   // rotation warps: CPR 16-byte chunks (8 pairs) per row of the first half,
   // RL row lanes, each thread ROT_ROWS rows of a tile at stride RL
@@ -70,8 +81,6 @@ struct Geo {
   static constexpr int ROT_ROWS = TK / RL;
   static constexpr int NENT = 2 * (ROT_ROWS - 1) + 2;  // offset-table entries
 };
-constexpr uint32_t TMEM_COLS = 64;  // S^T 0: [0,16), S^T 1: [16,32), O^T: [32,48)
-constexpr uint32_t COL_O = 32;
 constexpr int ERR_TIMEOUT = 16;
 // kind::f16, D fp32, A/B bf16, M = 128, N = 16; PV reads A (= V^T) MN-major
 constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
@@ -210,6 +219,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     }
     return;
   }
+  constexpr int TK = Geo<D>::TK;
   const int ntiles = (n + TK - 1) / TK;
   const int row0 = b * p.Lcap + kb;
   const int i = L - 1;
@@ -242,7 +252,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   }
   if (warp == WARP_MMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(su32(&tmem_slot)),
-                 "r"(TMEM_COLS));
+                 "r"(GG::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   fence_before();
@@ -289,10 +299,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
           const uint32_t ka = sbase + GG::OFF_K + sk * GG::TB;
           const uint32_t qa = sbase + GG::OFF_Q;
 #pragma unroll
-          for (int kk = 0; kk < GG::KSTEPS; ++kk) {
-            const uint32_t ko = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            const uint32_t qo = (kk >> 2) * (GG::QOPB / 2) + (kk & 3) * 32;
-            mma_ss(tmem + (uint32_t)((uq & 1) * 16), desc_k(ka + ko), desc_k(qa + qo), IDESC_QK, kk > 0 ? 1u : 0u);
+          for (int mb = 0; mb < TK / 128; ++mb) {  // keys 128 mb .. 128 mb + 127 (rows 128 B apart at D = 64)
+#pragma unroll
+            for (int kk = 0; kk < GG::KSTEPS; ++kk) {
+              const uint32_t ko = mb * 128 * 128 + (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+              const uint32_t qo = (kk >> 2) * (GG::QOPB / 2) + (kk & 3) * 32;
+              mma_ss(tmem + (uint32_t)((uq & 1) * GG::S_COLS + 16 * mb), desc_k(ka + ko), desc_k(qa + qo), IDESC_QK,
+                     kk > 0 ? 1u : 0u);
+            }
           }
           commit(&bar_sf[uq & 1]);
           commit(&bar_ke[sk]);
@@ -304,14 +318,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
           fence_after();
           const int sv = up % NVS;
           const uint32_t va = sbase + GG::OFF_V + sv * GG::TB;
-          const uint32_t pa = sbase + GG::OFF_P + (up & 1) * POPB;
+          const uint32_t pa = sbase + GG::OFF_P + (up & 1) * GG::POPB;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
+          for (int kk = 0; kk < TK / 16; ++kk) {
             // the second 64 rows of V^T: the tile's second box, or (D = 64)
             // the zero block, which lies after every V stage
             const uint32_t vk = va + kk * 2048;
             const uint32_t lbo = D == 128 ? (uint32_t)HALF_BYTES : sbase + (uint32_t)GG::OFF_Z - vk;
-            mma_ss(tmem + COL_O, desc_mn(vk, lbo), desc_k(pa + (kk >> 2) * (POPB / 2) + (kk & 3) * 32), IDESC_PV,
+            mma_ss(tmem + GG::COL_O, desc_mn(vk, lbo), desc_k(pa + (kk >> 2) * GG::PBOX + (kk & 3) * 32), IDESC_PV,
                    (up > 0 || kk > 0) ? 1u : 0u);
           }
           commit(&bar_ve[sv]);
@@ -482,7 +496,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     }
   } else {
     // ======================= softmax warpgroup =======================
-    const int r = threadIdx.x;  // key row of the tile / head-dim row of O^T / TMEM lane
+    const int r = threadIdx.x;  // key row of the tile (and r + 128 ..) / head-dim row of O^T / TMEM lane
+    constexpr int KPT = TK / 128;  // keys of a tile per thread
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const float sl2 = rsqrtf((float)D) * 1.4426950408889634f;
     // Q operand: rows h < GS hold the query heads, rows GS..15 zero; also zero
@@ -499,10 +514,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       }
       if (h >= GS)
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
+        for (int hf = 0; hf < TK / 64; ++hf)
 #pragma unroll
           for (int pb = 0; pb < 2; ++pb)
-            *reinterpret_cast<uint4 *>(gbase + GG::OFF_P + pb * POPB + hf * (POPB / 2) + op_off(h, c)) =
+            *reinterpret_cast<uint4 *>(gbase + GG::OFF_P + pb * GG::POPB + hf * GG::PBOX + op_off(h, c)) =
                 make_uint4(0u, 0u, 0u, 0u);
       if constexpr (D == 64) reinterpret_cast<uint4 *>(gbase + GG::OFF_Z)[r] = make_uint4(0u, 0u, 0u, 0u);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -522,18 +537,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       // where every warp of the group sees the abort and leaves together
       wait_b(&bar_sf[bsel], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT);
       fence_after();
-      uint32_t sr[8];
-      tmem_ld8(tmem + lane_base + (uint32_t)(bsel * 16), sr);
-      const int j = kb + u * TK + r;
-      const bool valid = j < ke;
-      float s[GS];
+      // keys r + 128 mb of the tile
+      float s[KPT][GS];
+      bool valid[KPT];
 #pragma unroll
-      for (int g = 0; g < GS; ++g) s[g] = valid ? __uint_as_float(sr[g]) * sl2 : -INFINITY;
+      for (int mb = 0; mb < KPT; ++mb) {
+        uint32_t sr[8];
+        tmem_ld8(tmem + lane_base + (uint32_t)(bsel * GG::S_COLS + 16 * mb), sr);
+        valid[mb] = kb + u * TK + 128 * mb + r < ke;
+#pragma unroll
+        for (int g = 0; g < GS; ++g) s[mb][g] = valid[mb] ? __uint_as_float(sr[g]) * sl2 : -INFINITY;
+      }
       // block-wide tile max per head
       float mt[GS];
 #pragma unroll
       for (int g = 0; g < GS; ++g) {
-        float x = s[g];
+        float x = s[0][g];
+#pragma unroll
+        for (int mb = 1; mb < KPT; ++mb) x = fmaxf(x, s[mb][g]);
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
         mt[g] = x;
@@ -571,34 +592,42 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
         wait_b(&bar_od, (u - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT);
         fence_after();
         uint32_t orow[8];
-        tmem_ld8(tmem + lane_base + COL_O, orow);
+        tmem_ld8(tmem + lane_base + GG::COL_O, orow);
 #pragma unroll
         for (int g = 0; g < GS; ++g) orow[g] = __float_as_uint(__uint_as_float(orow[g]) * f[g]);
-        tmem_st8(tmem + lane_base + COL_O, orow);
+        tmem_st8(tmem + lane_base + GG::COL_O, orow);
 #pragma unroll
         for (int g = 0; g < GS; ++g) l_part[g] *= f[g];
       }
       // P (bf16) into the B operand of the PV MMA: row g = head, column r = key
-      uint8_t *pbuf = gbase + GG::OFF_P + bsel * POPB + (r >> 6) * (POPB / 2);
-      const int chunk = (r & 63) >> 3;
 #pragma unroll
-      for (int g = 0; g < GS; ++g) {
-        const float pr = valid ? ex2(s[g] - m_run[g]) : 0.f;
-        l_part[g] += pr;
-        *reinterpret_cast<__nv_bfloat16 *>(pbuf + op_off(g, chunk) + (r & 7) * 2) = __float2bfloat16_rn(pr);
+      for (int mb = 0; mb < KPT; ++mb) {
+        const int kr = r + 128 * mb;  // key row of the tile: 64-key box kr / 64
+        uint8_t *pbuf = gbase + GG::OFF_P + bsel * GG::POPB + (kr >> 6) * GG::PBOX;
+        const int chunk = (kr & 63) >> 3;
+#pragma unroll
+        for (int g = 0; g < GS; ++g) {
+          const float pr = valid[mb] ? ex2(s[mb][g] - m_run[g]) : 0.f;
+          l_part[g] += pr;
+          *reinterpret_cast<__nv_bfloat16 *>(pbuf + op_off(g, chunk) + (kr & 7) * 2) = __float2bfloat16_rn(pr);
+        }
       }
       // a partial last tile: zero the V rows past the last key (the cache may
       // hold anything there, and 0 * NaN would poison the PV product)
       if (u == ntiles - 1 && (n % TK) != 0) {
         const int sv = u % NVS;
         wait_b(&bar_vf[sv], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT);
-        if (!valid && !abort_flag) {
+        if (!abort_flag) {
           uint8_t *vt = gbase + GG::OFF_V + sv * GG::TB;
 #pragma unroll
-          for (int hf = 0; hf < GG::NH; ++hf)
+          for (int mb = 0; mb < KPT; ++mb)
+            if (!valid[mb])
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4 *>(vt + hf * HALF_BYTES + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+              for (int hf = 0; hf < GG::NH; ++hf)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                  *reinterpret_cast<uint4 *>(vt + hf * HALF_BYTES + (r + 128 * mb) * 128 + c * 16) =
+                      make_uint4(0u, 0u, 0u, 0u);
         }
       }
       // last tile: PV of the previous tile must be complete before this
@@ -626,7 +655,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
     if (ok) {
       fence_after();
       uint32_t orow[8];
-      tmem_ld8(tmem + lane_base + COL_O, orow);
+      tmem_ld8(tmem + lane_base + GG::COL_O, orow);
       if (r < D)  // O^T row r is head_dim element r
 #pragma unroll
         for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * D + r] = __uint_as_float(orow[g]);
@@ -649,7 +678,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   __syncthreads();
   if (warp == WARP_MMA) {
     fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(GG::TMEM_COLS));
   }
 }
 
@@ -657,13 +686,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
 
 // ------------------------------------------------------------------ host
 // Split plan: one CTA per SM (the rings take ~200 KB of shared memory), one
-// wave of 148, whole 128-key tiles.
-void decode_tc_plan(int batch, int Hkv, int max_seqlen, int *nsplit, int *chunk) {
+// wave of 148, whole tiles (128 keys at head_dim 128, 256 at 64).
+void decode_tc_plan(int batch, int Hkv, int D, int max_seqlen, int *nsplit, int *chunk) {
   const long long bh = (long long)batch * (long long)Hkv;
   const int ns0 = bh >= 148 ? 1 : (int)(148 / max(1LL, bh));
   const int maxL = max(1, max_seqlen);
   int c = (maxL + ns0 - 1) / ns0;
-  c = (c + dtc::TK - 1) / dtc::TK * dtc::TK;
+  const int tk = D == 64 ? dtc::tile_keys<64>() : dtc::tile_keys<128>();
+  c = (c + tk - 1) / tk * tk;
   *chunk = c;
   *nsplit = (maxL + c - 1) / c;
 }
