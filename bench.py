@@ -294,6 +294,41 @@ def measure_extras(jl, dev, peaks, clocks_cls, local):
             "kcycles_per_tok": bi * mhz / 1e3 if mhz else None,
             "plain_kcycles_per_tok": pl * mhz / 1e3 if mhz else None, "clock_reasons": c.get("reasons")}
         del kc, vc
+    # batched decode with ragged lengths (uniform in [cap / 8, cap]), 32/8
+    # heads, head_dim 128; 20 steps replayed from a CUDA graph
+    for B, cap in ((8, 32768), (32, 8192)):
+        gd = torch.Generator(device=dev).manual_seed(B)
+        lens = torch.randint(cap // 8, cap + 1, (B,), generator=torch.Generator().manual_seed(B)).tolist()
+        kc = torch.randn(B, cap, 8, 128, generator=gd, device=dev, dtype=torch.bfloat16)
+        vc = torch.randn(B, cap, 8, 128, generator=gd, device=dev, dtype=torch.bfloat16)
+        qd = torch.randn(B, 32, 128, generator=gd, device=dev, dtype=torch.bfloat16)
+        sl = torch.tensor(lens, dtype=torch.int32, device=dev)
+        od = torch.empty_like(qd)
+        ws = torch.zeros(jl.jl_bifocal_decode_workspace_size(B, 32, 8, 128, cap), dtype=torch.uint8, device=dev)
+        res = {}
+        for lab, fl in (("bifocal", 0), ("plain", jl.JL_FLAG_PLAIN_CAUSAL)):
+            call = lambda: jl.jl_bifocal_decode(qd, kc, vc, sl, cap, 4096, 1024, 1e6, out=od, flags=fl,
+                                                workspace=ws)
+            s_ = torch.cuda.Stream()
+            s_.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(s_):
+                call()
+            torch.cuda.current_stream().wait_stream(s_)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(20):
+                    call()
+            res[lab] = statistics.median(_median_ms(graph.replay, 1) for _ in range(5)) * 1e3 / 20
+            del graph
+        nbytes = sum(2 * L * 8 * 128 * 2 for L in lens)
+        gbs = nbytes / res["bifocal"] / 1e3
+        ex[f"decode_ragged_b{B}"] = {
+            "workload": f"one decode step of {B} sequences, lengths uniform in [{cap // 8}, {cap}] (seeded), "
+                        "32/8 heads, head_dim 128, w_pre 4096, w0 1024 (20 steps from a CUDA graph)",
+            "us_per_step": res["bifocal"], "hbm_gbs": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "plain_us_per_step": res["plain"], "plain_hbm_gbs": nbytes / res["plain"] / 1e3}
+        del kc, vc
     return ex
 
 

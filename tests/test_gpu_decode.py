@@ -184,3 +184,48 @@ def test_decode_replays_from_a_cuda_graph():
         assert_close(to_np(out), ro, torch.bfloat16, f"out step {step}")
         assert_close(to_np(lse), rl, torch.bfloat16, f"lse step {step}")
     assert int(ws[:4].view(torch.int32).item()) == 0
+
+
+BALANCE = [
+    # (seqlens, Hq, Hkv, D): fewer (sequence, kv head) pairs than SMs put the
+    # splits on the device-planned balanced layout (one unit per SM)
+    ((0, 1, 129, 5000, 20000, 7, 12345, 256), 32, 8, 128),     # empty, tiny and long sequences
+    ((0, 1, 129, 5000, 20000, 7, 12345, 256), 32, 8, 64),
+    (tuple(range(300, 300 + 18 * 700, 700)), 16, 8, 128),      # 144 pairs: one unit per pair
+    (tuple(range(50, 50 + 37 * 97, 97)), 16, 4, 128),          # 148 pairs: the (split, head, sequence) grid
+    ((3000,) * 5 + (1,), 8, 1, 128),                           # one kv head: up to 148 units
+]
+
+
+@pytest.mark.parametrize("seqlens,Hq,Hkv,D", BALANCE)
+def test_decode_balanced_splits(seqlens, Hq, Hkv, D):
+    # every key of every (sequence, kv head) falls in exactly one unit: the
+    # combined result matches the oracle for ragged lengths, and repeated
+    # calls with other lengths in the same workspace stay correct
+    B, cap = len(seqlens), max(seqlens)
+    g = torch.Generator().manual_seed(B * 1000 + D)
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16)
+    kc = torch.randn(B, cap, Hkv, D, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, cap, Hkv, D, generator=g).to(torch.bfloat16)
+    for lens in (list(seqlens), [max(0, x - 129) for x in reversed(seqlens)]):
+        out, lse = decode_gpu(q, kc, vc, lens, cap, 3000, 500, 1e6)
+        ro, rl = oracle.bifocal_decode(q, kc, vc, lens, 3000, 500, 1e6)
+        assert_close(to_np(out), ro, torch.bfloat16, f"out {lens[:3]}")
+        assert_close(to_np(lse), rl, torch.bfloat16, f"lse {lens[:3]}")
+
+
+@pytest.mark.parametrize("Hkv,D,dtype", [(2, 128, torch.bfloat16), (2, 64, torch.bfloat16),
+                                         (2, 128, torch.float32), (80, 128, torch.bfloat16)])
+def test_decode_length_past_max_seqlen_writes_zero(Hkv, D, dtype):
+    # a length above max_seqlen (within the cache) is outside the contract:
+    # zeros and LSE -inf, on every decode kernel and split plan (80 kv heads x
+    # 2 sequences is past one unit per SM: the per-split grid)
+    g = torch.Generator().manual_seed(Hkv + D)
+    q = torch.randn(2, 2 * Hkv, D, generator=g).to(dtype)
+    kc = torch.randn(2, 100, Hkv, D, generator=g).to(dtype)
+    vc = torch.randn(2, 100, Hkv, D, generator=g).to(dtype)
+    out, lse = decode_gpu(q, kc, vc, [50, 90], 60, 30, 8, 1e4)
+    assert torch.all(out[1] == 0) and torch.all(torch.isinf(lse[1]))
+    ro, rl = oracle.bifocal_decode(q[:1], kc[:1], vc[:1], [50], 30, 8, 1e4)
+    assert_close(to_np(out[:1]), ro, dtype, "row 0")
+    assert_close(to_np(lse[:1]), rl, dtype, "row 0 lse")

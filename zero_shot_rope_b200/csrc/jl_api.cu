@@ -20,10 +20,11 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(int batch, int Hq, int Hkv, int D, int max_seqlen, int elem);
 size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen);
+size_t decode_plan_tab_bytes();
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
                           const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
                           long long w_pre, int w0, int window, const InvFreq &inv, int plain, float *part_o,
-                          float *part_ml, int *err, void *out, float *lse, cudaStream_t st);
+                          float *part_ml, int2 *plan_tab, int *err, void *out, float *lse, cudaStream_t st);
 size_t tc_prefill_workspace(int batch, int T_total, int Hq, int Hkv, int D, uint32_t flags);
 cudaError_t launch_tc_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
                               const int32_t *cu, const int32_t *cu_k, int batch, int T_total, int Tk,
@@ -204,7 +205,8 @@ size_t jl_bifocal_decode_workspace_size(int32_t batch, int32_t n_q_heads, int32_
   if (n_q_heads % n_kv_heads != 0) return 0;
   // one layout serves every dtype and both decode kernels
   const size_t rows = jl::decode_partial_rows(batch, n_q_heads, n_kv_heads, head_dim, max_seqlen);
-  return 256 + align256(rows * head_dim * sizeof(float)) + align256(rows * 2 * sizeof(float));
+  return 256 + align256(rows * head_dim * sizeof(float)) + align256(rows * 2 * sizeof(float)) +
+         align256(jl::decode_plan_tab_bytes());
 }
 
 jl_status jl_bifocal_decode_window(const void *q, const void *k_cache, const void *v_cache,
@@ -244,13 +246,14 @@ jl_status jl_bifocal_decode_window(const void *q, const void *k_cache, const voi
   int *err = (int *)workspace;
   float *part_o = (float *)((char *)workspace + 256);
   float *part_ml = (float *)((char *)workspace + 256 + align256(rows * head_dim * sizeof(float)));
+  int2 *plan_tab = (int2 *)((char *)part_ml + align256(rows * 2 * sizeof(float)));
   const jl::InvFreq inv = make_inv_freq(head_dim, rope_theta);
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), st);
   if (e == cudaSuccess)
     e = jl::launch_decode(dtype == JL_BF16, head_dim, gs, q, k_cache, v_cache, seqlens, batch, cache_capacity,
                           max_seqlen, n_q_heads, n_kv_heads, w_pretrained, w0, window, inv,
-                          (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0, part_o, part_ml, err, out, lse, st);
+                          (flags & JL_FLAG_PLAIN_CAUSAL) ? 1 : 0, part_o, part_ml, plan_tab, err, out, lse, st);
   return e == cudaSuccess ? ok() : cuda_fail(e, "decode launch");
 }
 

@@ -24,6 +24,8 @@
 //    rows; the slots are merged at the end, the splits by a second kernel
 //    (the LSE merge of §2 "Mesclagem ... Inclusão–Exclusão" applied to key
 //    ranges).
+#include <algorithm>
+
 #include "jl_common.cuh"
 #include "jl_ptx.cuh"
 
@@ -110,6 +112,7 @@ struct DecodeArgs {
   long long w_pre;
   int w0, plain, chunk, nsplit;
   int window;  // sliding-window width (0: none)
+  int max_seqlen;
   float *part_o, *part_ml;
   int *err;
 };
@@ -132,10 +135,10 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap mK, const __grid_const
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, slot = tid / TPR, t = tid % TPR;
   int L = p.seqlens[b];
-  // a length outside [0, Lcap], or with more keys than the planned splits
-  // hold, attends to nothing rather than reading past the cache; a
-  // sliding-window layer sees keys jw .. L-1 only
-  if (L < 0 || L > p.Lcap) L = 0;
+  // a length outside [0, min(Lcap, max_seqlen)], or with more keys than the
+  // planned splits hold, attends to nothing rather than reading past the
+  // cache; a sliding-window layer sees keys jw .. L-1 only
+  if (L < 0 || L > p.Lcap || L > p.max_seqlen) L = 0;
   int jw = p.window > 0 ? max(0, L - p.window) : 0;
   if (L - jw > p.nsplit * p.chunk) L = jw = 0;
   const int kb = jw + split * p.chunk;
@@ -360,19 +363,32 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap mK, const __grid_const
 template <typename T, int D>
 __global__ void __launch_bounds__(D)
 decode_combine_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml, int nsplit,
-                      T *__restrict__ out, float *__restrict__ lse) {
+                      const int2 *__restrict__ plan_tab, int GS, int Hkv, T *__restrict__ out,
+                      float *__restrict__ lse) {
   const int bh = blockIdx.x, d = threadIdx.x;
-  const float *ml = part_ml + (size_t)bh * nsplit * 2;
+  // rows of this (sequence, head)'s splits: row0 + s * stride, s < ns.  With
+  // a balanced plan the rows are per unit (GS heads each) and the plan's
+  // table gives the sequence's first unit and units per kv head.
+  size_t row0 = (size_t)bh * nsplit, stride = 1;
+  int ns = nsplit;
+  if (plan_tab != nullptr) {
+    const int Hq = GS * Hkv, b = bh / Hq, h = bh % Hq;
+    const int2 e = plan_tab[b];
+    ns = e.y;
+    row0 = ((size_t)e.x + (size_t)(h / GS) * ns) * GS + h % GS;
+    stride = GS;
+  }
   float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, ml[2 * s]);
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, part_ml[(row0 + s * stride) * 2]);
   float acc = 0.f, l = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float m = ml[2 * s];
+    for (int s = 0; s < ns; ++s) {
+      const size_t row = row0 + s * stride;
+      const float m = part_ml[row * 2];
       if (m == -INFINITY) continue;
       const float w = exp2f(m - M);
-      l = fmaf(w, ml[2 * s + 1], l);
-      acc = fmaf(w, part_o[((size_t)bh * nsplit + s) * D + d], acc);
+      l = fmaf(w, part_ml[row * 2 + 1], l);
+      acc = fmaf(w, part_o[row * D + d], acc);
     }
   }
   out[(size_t)bh * D + d] = from_f<T>(l > 0.f ? acc / l : 0.f);
@@ -445,7 +461,8 @@ static cudaError_t launch_decode_t(const CUtensorMap &mK, const CUtensorMap &mV,
   dim3 grid(pl.nsplit, a.Hkv, B);
   kern<<<grid, DEC_THREADS, pl.smem_bytes, st>>>(mK, mV, a, inv);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  decode_combine_kernel<T, D><<<B * a.Hq, D, 0, st>>>(a.part_o, a.part_ml, pl.nsplit, (T *)out, lse);
+  decode_combine_kernel<T, D><<<B * a.Hq, D, 0, st>>>(a.part_o, a.part_ml, pl.nsplit, nullptr, 1, 1, (T *)out,
+                                                      lse);
   return cudaGetLastError();
 }
 
@@ -464,9 +481,10 @@ static cudaError_t launch_decode_d(int GS, const CUtensorMap &mK, const CUtensor
 
 void decode_tc_plan(int batch, int Hkv, int D, int max_seqlen, int *nsplit, int *chunk);
 cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
-                             const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                             int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
-                             float *part_ml, int *err, cudaStream_t st);
+                             const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
+                             long long w_pre, int w0, int window, const InvFreq &inv, int plain, int nsplit,
+                             int chunk, float *part_o, float *part_ml, int2 *plan_tab, __nv_bfloat16 *out,
+                             float *lse, int *err, cudaStream_t st);
 
 static bool use_tc_decode(bool bf16, int D, int GS) { return bf16 && (D == 128 || D == 64) && GS <= 8; }
 
@@ -481,8 +499,16 @@ size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
   const int tiles64 = (max(1, max_seqlen) + DEC_TK - 1) / DEC_TK;
   int ns = min(max(1, 2 * 148 / per_bh), tiles64);  // both element sizes of decode_plan
   if (use_tc_decode(true, D, GS)) ns = max(ns, min(max(1, 148 / per_bh), (max(1, max_seqlen) + 127) / 128));
-  return (size_t)batch * Hq * ns;
+  size_t rows = (size_t)batch * Hq * ns;
+  // the tensor-core decode's balanced plan: at most one unit of GS rows per SM
+  if (use_tc_decode(true, D, GS) && per_bh < 148) rows = std::max(rows, (size_t)148 * GS);
+  return rows;
 }
+
+// Whether the tensor-core decode plans its splits on the device (fewer
+// (sequence, kv head) pairs than SMs), and the bytes of that plan's table.
+static bool decode_tc_balanced(int batch, int Hkv) { return sequence_heads(batch, Hkv) < 148; }
+size_t decode_plan_tab_bytes() { return 148 * sizeof(int2); }
 
 static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv, int D) {
   // bf16 cache viewed as (d, head, row); 64 x 1 x (keys of a tile) boxes,
@@ -501,7 +527,7 @@ static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv, i
 cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *kc, const void *vc,
                           const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
                           long long w_pre, int w0, int window, const InvFreq &inv, int plain, float *part_o,
-                          float *part_ml, int *err, void *out, float *lse, cudaStream_t st) {
+                          float *part_ml, int2 *plan_tab, int *err, void *out, float *lse, cudaStream_t st) {
   const int elem = bf16 ? 2 : 4;
   // the splits cover at most `window` keys per sequence
   const int keys = window > 0 ? min(max_seqlen, window) : max_seqlen;
@@ -511,15 +537,17 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
       return cudaErrorInvalidValue;
     int ns, chunk;
     decode_tc_plan(B, Hkv, D, keys, &ns, &chunk);
-    cudaError_t e = launch_decode_tc(GS, D, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, Hq, Hkv, w_pre, w0,
-                                     window, inv, plain, ns, chunk, part_o, part_ml, err, st);
+    int2 *tab = decode_tc_balanced(B, Hkv) ? plan_tab : nullptr;
+    cudaError_t e = launch_decode_tc(GS, D, tK, tV, (const __nv_bfloat16 *)q, seqlens, B, Lcap, max_seqlen, Hq, Hkv,
+                                     w_pre, w0, window, inv, plain, ns, chunk, part_o, part_ml, tab,
+                                     (__nv_bfloat16 *)out, lse, err, st);
     if (e != cudaSuccess) return e;
     if (D == 128)
-      decode_combine_kernel<__nv_bfloat16, 128><<<B * Hq, 128, 0, st>>>(part_o, part_ml, ns,
+      decode_combine_kernel<__nv_bfloat16, 128><<<B * Hq, 128, 0, st>>>(part_o, part_ml, ns, tab, GS, Hkv,
                                                                         (__nv_bfloat16 *)out, lse);
     else
-      decode_combine_kernel<__nv_bfloat16, 64><<<B * Hq, 64, 0, st>>>(part_o, part_ml, ns, (__nv_bfloat16 *)out,
-                                                                      lse);
+      decode_combine_kernel<__nv_bfloat16, 64><<<B * Hq, 64, 0, st>>>(part_o, part_ml, ns, tab, GS, Hkv,
+                                                                      (__nv_bfloat16 *)out, lse);
     return cudaGetLastError();
   }
   const DecodePlan pl = decode_plan(B, Hq, Hkv, D, keys, elem);
@@ -536,6 +564,7 @@ cudaError_t launch_decode(bool bf16, int D, int GS, const void *q, const void *k
   a.w0 = w0;
   a.plain = plain;
   a.window = window;
+  a.max_seqlen = max_seqlen;
   a.chunk = pl.chunk;
   a.nsplit = pl.nsplit;
   a.part_o = part_o;

@@ -95,7 +95,125 @@ struct Args {
   int window;  // sliding-window width (0: none)
   float *part_o, *part_ml;
   int *err;
+  // balanced plan (fewer (sequence, kv head) pairs than SMs): one CTA per
+  // SM, units sized on the device from the lengths; CTA 0 writes per
+  // sequence (first unit, units per kv head) for the combine
+  int balanced, batch, max_seqlen;
+  int2 *plan_tab;
+  // outputs, for the sequences with no key under the balanced plan
+  __nv_bfloat16 *out;
+  float *lse;
 };
+
+constexpr int NSM = 148;
+
+// The balanced plan, computed by one warp of every CTA from the lengths on
+// the device (so a captured step replays correctly).  Sequence b attends to
+// n_b keys, t_b = ceil(n_b / TK) tiles; a unit is up to k tiles of one
+// (sequence, kv head), so (sequence b, kv head) splits into ceil(t_b / k)
+// units.  k is the smallest tile count whose units fit one wave (sum over b
+// of Hkv * ceil(t_b / k) <= NSM): the longest unit, which sets the step
+// time, is then as short as one wave allows.  The warp tests 32 candidate
+// k at once and narrows the range until one is left.  Units are numbered
+// sequence-major, then kv head, then split.  plan_s receives (b, kv head,
+// split, keys per unit, L_b, first key) of this CTA's unit, or b = -1; CTA 0
+// writes (first unit, units per kv head) of every sequence to the table (the
+// combine's map) and the output of every sequence with no key (zeros, LSE
+// -inf).  s_t, s_L, s_jw: NSM ints of shared memory each.  Out of line, so
+// that the kernel's loops stay compact.  Requires B * Hkv < NSM (B < NSM).
+__device__ __noinline__ void plan_balanced(const Args &p, int TK, int D, int lane, int *plan_s, int *s_t, int *s_L,
+                                           int *s_jw) {
+  const unsigned full = 0xffffffffu;
+  const int B = p.batch;
+  int T = 0, nne = 0, tmax = 0;
+#pragma unroll 1
+  for (int b = lane; b < B; b += 32) {
+    int L = p.seqlens[b];
+    if (L < 0 || L > p.Lcap || L > p.max_seqlen) L = 0;  // outside the contract: no key
+    const int jw = p.window > 0 ? max(0, L - p.window) : 0;
+    const int t = (L - jw + TK - 1) / TK;
+    s_t[b] = t;
+    s_L[b] = L;
+    s_jw[b] = jw;
+    T += t;
+    nne += t > 0 ? 1 : 0;
+    tmax = max(tmax, t);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    T += __shfl_xor_sync(full, T, o);
+    nne += __shfl_xor_sync(full, nne, o);
+    tmax = max(tmax, __shfl_xor_sync(full, tmax, o));
+  }
+  __syncwarp();
+  const int S = NSM / p.Hkv;  // units per kv head in one wave (>= B >= nne)
+  int k = 1;
+  if (T > 0) {
+    // below ceil(T / S) the units exceed S; at hi they fit: either
+    // sum(t_b / k + 1) <= S, or k = tmax (one unit per sequence)
+    int hi = S > nne ? (T + (S - nne) - 1) / (S - nne) : tmax;
+    hi = min(max(hi, 1), tmax);
+    int lo = min(max((T + S - 1) / S, 1), hi);
+#pragma unroll 1
+    while (lo < hi) {
+      // candidates nondecreasing over the lanes, the last one hi
+      const int step = (hi - lo + 30) / 31;
+      const int kc = min(lo + step * lane, hi);
+      int units = 0;
+#pragma unroll 1
+      for (int b = 0; b < B; ++b) units += (s_t[b] + kc - 1) / kc;
+      const unsigned fits = __ballot_sync(full, units <= S);  // a suffix of the lanes, lane 31 included
+      const int f = __ffs(fits) - 1;
+      const int kf = __shfl_sync(full, kc, f);
+      const int kp = __shfl_sync(full, kc, f > 0 ? f - 1 : 0);
+      lo = min(f > 0 ? kp + 1 : lo, kf);
+      hi = kf;
+    }
+    k = lo;
+  }
+  // locate this CTA's unit: exclusive prefix of Hkv * ceil(t_b / k) over b
+  const int u = blockIdx.x;
+  if (lane == 0) plan_s[0] = -1;
+  __syncwarp();
+  int carry = 0;
+#pragma unroll 1
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
+    const int ns = b < B ? (s_t[b] + k - 1) / k : 0;
+    int inc = ns * p.Hkv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    const int base = carry + inc - ns * p.Hkv;  // exclusive
+    if (b < B) {
+      if (u == 0) p.plan_tab[b] = make_int2(base, ns);
+      if (ns > 0 && u >= base && u < base + ns * p.Hkv) {
+        const int kvh = (u - base) / ns;
+        plan_s[0] = b;
+        plan_s[1] = kvh;
+        plan_s[2] = u - base - kvh * ns;
+        plan_s[3] = k * TK;
+        plan_s[4] = s_L[b];
+        plan_s[5] = s_jw[b];
+      }
+    }
+    carry += __shfl_sync(full, inc, 31);
+  }
+  if (u == 0) {
+    // sequences with no key: no unit writes them
+#pragma unroll 1
+    for (int b = 0; b < B; ++b) {
+      if (s_t[b] == 0) {
+        uint4 *o4 = reinterpret_cast<uint4 *>(p.out + (size_t)b * p.Hq * D);
+        for (int idx = lane; idx < p.Hq * D / 8; idx += 32) o4[idx] = make_uint4(0u, 0u, 0u, 0u);
+        if (p.lse != nullptr)
+          for (int h = lane; h < p.Hq; h += 32) p.lse[(size_t)b * p.Hq + h] = -INFINITY;
+      }
+    }
+  }
+}
 
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -199,33 +317,40 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
   __shared__ float4 otab[Geo<D>::NENT][2][16];
 
   using GG = Geo<D>;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  int L = p.seqlens[b];
-  if (L < 0 || L > p.Lcap) L = 0;  // never read past the cache
-  // a sliding-window layer sees keys jw .. L-1 only; the splits cover them
-  int jw = p.window > 0 ? max(0, L - p.window) : 0;
-  if (L - jw > p.nsplit * p.chunk) L = jw = 0;  // more keys than the planned splits hold
-  const int kb = jw + split * p.chunk;
-  const int ke = min(L, kb + p.chunk);
-  const int n = max(0, ke - kb);
-  const size_t pidx = ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;  // + g * nsplit
-  if (n == 0) {
-    for (int idx = threadIdx.x; idx < GS * D; idx += THREADS)
-      p.part_o[(pidx + (size_t)(idx / D) * p.nsplit) * D + idx % D] = 0.f;
-    if (threadIdx.x < GS) {
-      p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 0] = -INFINITY;
-      p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 1] = 0.f;
-    }
-    return;
-  }
   constexpr int TK = Geo<D>::TK;
-  const int ntiles = (n + TK - 1) / TK;
-  const int row0 = b * p.Lcap + kb;
-  const int i = L - 1;
-  const int G = p.plain ? 1 : (int)group_size(L, p.w_pre);
-  const bool bif = G > 1;
-  const int j_local = (int)max(0LL, (long long)L - (long long)p.w0);  // keys >= j_local are local
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this CTA's (sequence, kv head, split, keys per split, length, first
+  // key): from the grid, or (balanced) from the plan; read back from shared
+  // memory by every role
+  __shared__ int plan_s[6];
+  __shared__ int s_t[NSM], s_L[NSM], s_jw[NSM];
+  if (!p.balanced) {
+    const int split = blockIdx.x, chunk = p.chunk;
+    int L = p.seqlens[blockIdx.z];
+    if (L < 0 || L > p.Lcap || L > p.max_seqlen) L = 0;  // outside the contract: no key
+    // a sliding-window layer sees keys jw .. L-1 only; the splits cover them
+    int jw = p.window > 0 ? max(0, L - p.window) : 0;
+    if (L - jw > p.nsplit * chunk) L = jw = 0;  // more keys than the planned splits hold
+    if (jw + split * chunk >= L) {
+      // no key in this split: an empty partial
+      const size_t pidx = ((size_t)blockIdx.z * p.Hq + (size_t)blockIdx.y * GS) * p.nsplit + split;
+      for (int idx = threadIdx.x; idx < GS * D; idx += THREADS)
+        p.part_o[(pidx + (size_t)(idx / D) * p.nsplit) * D + idx % D] = 0.f;
+      if (threadIdx.x < GS) {
+        p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 0] = -INFINITY;
+        p.part_ml[(pidx + (size_t)threadIdx.x * p.nsplit) * 2 + 1] = 0.f;
+      }
+      return;
+    }
+    if (threadIdx.x == 0) {
+      plan_s[0] = blockIdx.z;
+      plan_s[1] = blockIdx.y;
+      plan_s[2] = split;
+      plan_s[3] = chunk;
+      plan_s[4] = L;
+      plan_s[5] = jw;
+    }
+  }
 
   const uint32_t sbase = (su32(smem_raw) + 1023u) & ~1023u;
   uint8_t *gbase = smem_raw + (sbase - su32(smem_raw));
@@ -255,10 +380,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
                  "r"(GG::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
+  // the balanced plan runs on a rotation warp beside the set-up above
+  if (p.balanced && warp == 4) plan_balanced(p, TK, D, lane, plan_s, s_t, s_L, s_jw);
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem = tmem_slot;
+  if (plan_s[0] < 0) {  // balanced plan: no unit for this CTA (uniform)
+    if (warp == WARP_MMA)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(GG::TMEM_COLS));
+    return;
+  }
+  const int b = plan_s[0], kvh = plan_s[1], split = plan_s[2], chunk = plan_s[3], L = plan_s[4], jw = plan_s[5];
+  const int kb = jw + split * chunk;
+  const int ke = min(L, kb + chunk);
+  const int n = ke - kb;  // >= 1
+  // partial rows of this CTA's heads g: pidx + g * pstride (balanced: the
+  // unit's GS rows; otherwise (sequence, head, split) with nsplit splits)
+  const size_t pidx = p.balanced ? (size_t)blockIdx.x * GS
+                                 : ((size_t)b * p.Hq + (size_t)kvh * GS) * p.nsplit + split;
+  const size_t pstride = p.balanced ? 1 : (size_t)p.nsplit;
+  const int ntiles = (n + TK - 1) / TK;
+  const int row0 = b * p.Lcap + kb;
+  const int i = L - 1;
+  const int G = p.plain ? 1 : (int)group_size(L, p.w_pre);
+  const bool bif = G > 1;
+  const int j_local = (int)max(0LL, (long long)L - (long long)p.w0);  // keys >= j_local are local
+
 
   if (warp == WARP_TMA) {
     // ======================= TMA producer =======================
@@ -658,18 +806,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__
       tmem_ld8(tmem + lane_base + GG::COL_O, orow);
       if (r < D)  // O^T row r is head_dim element r
 #pragma unroll
-        for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * D + r] = __uint_as_float(orow[g]);
+        for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * pstride) * D + r] = __uint_as_float(orow[g]);
       if (r < GS) {
         const float l = lred[0][r] + lred[1][r] + lred[2][r] + lred[3][r];
-        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 0] = m_run[r];
-        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 1] = l;
+        p.part_ml[(pidx + (size_t)r * pstride) * 2 + 0] = m_run[r];
+        p.part_ml[(pidx + (size_t)r * pstride) * 2 + 1] = l;
       }
     } else {
       if (r < D)
-        for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * p.nsplit) * D + r] = 0.f;
+        for (int g = 0; g < GS; ++g) p.part_o[(pidx + (size_t)g * pstride) * D + r] = 0.f;
       if (r < GS) {
-        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 0] = -INFINITY;
-        p.part_ml[(pidx + (size_t)r * p.nsplit) * 2 + 1] = 0.f;
+        p.part_ml[(pidx + (size_t)r * pstride) * 2 + 0] = -INFINITY;
+        p.part_ml[(pidx + (size_t)r * pstride) * 2 + 1] = 0.f;
       }
     }
   }
@@ -699,9 +847,10 @@ void decode_tc_plan(int batch, int Hkv, int D, int max_seqlen, int *nsplit, int 
 }
 
 cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtensorMap &mV, const __nv_bfloat16 *q,
-                             const int32_t *seqlens, int B, int Lcap, int Hq, int Hkv, long long w_pre, int w0,
-                             int window, const InvFreq &inv, int plain, int nsplit, int chunk, float *part_o,
-                             float *part_ml, int *err, cudaStream_t st) {
+                             const int32_t *seqlens, int B, int Lcap, int max_seqlen, int Hq, int Hkv,
+                             long long w_pre, int w0, int window, const InvFreq &inv, int plain, int nsplit,
+                             int chunk, float *part_o, float *part_ml, int2 *plan_tab, __nv_bfloat16 *out,
+                             float *lse, int *err, cudaStream_t st) {
   dtc::Args a;
   a.q = q;
   a.seqlens = seqlens;
@@ -717,7 +866,14 @@ cudaError_t launch_decode_tc(int GS, int D, const CUtensorMap &mK, const CUtenso
   a.part_o = part_o;
   a.part_ml = part_ml;
   a.err = err;
-  dim3 grid(nsplit, Hkv, B);
+  // balanced: one CTA per SM, units planned on the device
+  a.balanced = plan_tab != nullptr;
+  a.batch = B;
+  a.max_seqlen = max_seqlen;
+  a.plan_tab = plan_tab;
+  a.out = out;
+  a.lse = lse;
+  const dim3 grid = a.balanced ? dim3(dtc::NSM, 1, 1) : dim3(nsplit, Hkv, B);
   cudaError_t e;
 #define JL_DTC(GG, DD)                                                                                    \
   e = cudaFuncSetAttribute(dtc::decode_tc_kernel<GG, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
