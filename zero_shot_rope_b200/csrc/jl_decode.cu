@@ -505,9 +505,13 @@ size_t decode_partial_rows(int batch, int Hq, int Hkv, int D, int max_seqlen) {
   return rows;
 }
 
-// Whether the tensor-core decode plans its splits on the device (fewer
-// (sequence, kv head) pairs than SMs), and the bytes of that plan's table.
-static bool decode_tc_balanced(int batch, int Hkv) { return sequence_heads(batch, Hkv) < 148; }
+// Whether the tensor-core decode plans its splits on the device: for two or
+// more sequences (whose lengths may differ) in fewer (sequence, kv head)
+// pairs than SMs.  A single sequence keeps the host plan, sized by
+// max_seqlen: the device plan costs ~2 us per step, which only pays when
+// lengths differ (or the one length is well below max_seqlen).  Also the
+// bytes of the plan's table.
+static bool decode_tc_balanced(int batch, int Hkv) { return batch >= 2 && sequence_heads(batch, Hkv) < 148; }
 size_t decode_plan_tab_bytes() { return 148 * sizeof(int2); }
 
 static bool make_tile_map(CUtensorMap *m, const void *base, int rows, int Hkv, int D) {
