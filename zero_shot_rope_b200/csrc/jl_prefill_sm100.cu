@@ -94,18 +94,42 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
                    su32(bar))
                : "memory");
 }
-__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+// tcgen05.mma, kind::f16, D in TMEM: A and B from shared memory (ss) or A
+// from TMEM (ts).  The shared-memory descriptors come as 32-bit halves: the
+// low half (start address) varies by stage and k-step, the high half is
+// fixed, so the single issuing thread spends one add per operand per k-step.
+__device__ __forceinline__ void umma_ss_lh(uint32_t d, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi,
+                                           uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d),
+      "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc));
 }
-__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                        uint32_t acc) {
+template <uint32_t ACC>
+__device__ __forceinline__ void umma_ss_lhc(uint32_t d, uint32_t alo, uint32_t ahi, uint32_t blo, uint32_t bhi,
+                                            uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "mov.b64 da, {%1, %2};\n\tmov.b64 db, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d),
+      "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "n"(ACC));
+}
+template <uint32_t ACC>
+__device__ __forceinline__ void umma_ts_lhc(uint32_t d, uint32_t a_tmem, uint32_t blo, uint32_t bhi, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "n"(ACC));
+}
+__device__ __forceinline__ void umma_ts_lh(uint32_t d, uint32_t a_tmem, uint32_t blo, uint32_t bhi, uint32_t idesc,
+                                           uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "r"(blo), "r"(bhi), "r"(idesc), "r"(acc));
 }
 
 #define JL_R32(a) \
@@ -620,17 +644,24 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
       bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
       bool qg_seen = false;
       int v = 0;
+      // descriptor halves: the start address field (addr >> 4, 14 bits) of
+      // every stage and k-step stays below 2^14, so a stage or a k-step adds
+      // to the low half only; the high halves are fixed
+      const uint64_t vd0 = desc_mn_sw128(sbase + OFF_V1, HALF_BYTES);
+      const uint32_t v0lo = (uint32_t)vd0, vhi = (uint32_t)(vd0 >> 32);
+      const uint64_t kd0 = desc_k_sw128(sbase + OFF_K1);
+      const uint32_t k0lo = (uint32_t)kd0, dhi = (uint32_t)(kd0 >> 32);
+      const uint32_t qlo_b = (uint32_t)desc_k_sw128(sbase + OFF_Q), qlo_g = (uint32_t)desc_k_sw128(sbase + GG::P1_OFF_QG);
       auto issue_pv = [&](int u) -> bool {
         const int vs_ = u % NVS;
         if (!wait_b(&bar_vf[vs_], (u / NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         if (!wait_b(&bar_pr[u & 1], (u >> 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t vaddr = sbase + OFF_V1 + vs_ * GG::TB;
+        const uint32_t vlo = v0lo + (uint32_t)vs_ * (uint32_t)(GG::TB >> 4);
         const uint32_t pcol = tmem + (uint32_t)((u & 1) * 128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + COL_O, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), GG::IDESC_PV,
-                  (u > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_lh(tmem + COL_O, pcol + kk * 8, vlo + kk * 128, vhi, GG::IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&bar_ve[vs_]);
         umma_commit(&bar_od);
         return true;
@@ -649,13 +680,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_cons
         uint64_t *kready = kcorr ? &bar_kr[st] : &bar_kf[st];
         if (!(ok = wait_b(kready, (v / P1_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))) break;
         tc_fence_after();
-        const uint32_t qaddr = sbase + (vx.grp ? GG::P1_OFF_QG : OFF_Q);
-        const uint32_t kaddr = sbase + OFF_K1 + st * GG::TB;
+        const uint32_t qlo = vx.grp ? qlo_g : qlo_b;
+        const uint32_t kdlo = k0lo + (uint32_t)st * (uint32_t)(GG::TB >> 4);
         const uint32_t scol = tmem + (uint32_t)((v & 1) * 128);
 #pragma unroll
         for (int kk = 0; kk < GG::KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss_lh(scol, qlo + off, dhi, kdlo + off, dhi, IDESC_QK, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bar_sf[v & 1]);
         umma_commit(&bar_ke[st]);
@@ -1077,6 +1108,13 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       // head's PV runs.  S_x is reused by QK_x(v+1) only after PV_x(v) (which
       // read P_x(v) from it) has been issued.
       bool ok = wait_b(&bar_q, 0, &abort_flag, p.err, ERR_TIMEOUT_MMA);
+      // descriptor halves: the start address field (addr >> 4, 14 bits) of
+      // every stage and k-step stays below 2^14, so a stage or a k-step adds
+      // to the low half only; the high halves are fixed
+      const uint64_t qd0 = desc_k_sw128(sbase + P2_OFF_Q), vd0 = desc_mn_sw128(sbase + GG::OFF_V, HALF_BYTES);
+      const uint32_t q0lo = (uint32_t)qd0, q1lo = q0lo + (uint32_t)(GG::TB >> 4), dhi = (uint32_t)(qd0 >> 32);
+      const uint32_t k0lo = (uint32_t)desc_k_sw128(sbase + GG::OFF_K);
+      const uint32_t v0lo = (uint32_t)vd0, vhi = (uint32_t)(vd0 >> 32);
       auto issue_qk = [&](int x, int v) -> bool {
         // the first grouped QK of a head reads its query tile rotated in
         // place by that head's softmax warpgroup
@@ -1088,13 +1126,13 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
           if (!wait_b(kready, (v / P2_NKS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         }
         tc_fence_after();
-        const uint32_t qaddr = sbase + P2_OFF_Q + x * GG::TB;
-        const uint32_t kaddr = sbase + GG::OFF_K + (v % P2_NKS) * GG::TB;
         const uint32_t scol = tmem + (uint32_t)(x * 128);
+        const uint32_t qlo = x ? q1lo : q0lo, kdlo = k0lo + (uint32_t)(v % P2_NKS) * (uint32_t)(GG::TB >> 4);
+        umma_ss_lhc<0>(scol, qlo, dhi, kdlo, dhi, IDESC_QK);
 #pragma unroll
-        for (int kk = 0; kk < GG::KSTEPS; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          umma_ss(scol, desc_k_sw128(qaddr + off), desc_k_sw128(kaddr + off), IDESC_QK, kk > 0 ? 1u : 0u);
+        for (int kk = 1; kk < GG::KSTEPS; ++kk) {
+          const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+          umma_ss_lhc<1>(scol, qlo + off, dhi, kdlo + off, dhi, IDESC_QK);
         }
         umma_commit(&bar_sf[x]);
         if (x == 1) umma_commit(&bar_ke[v % P2_NKS]);  // both heads' QK issued
@@ -1104,21 +1142,21 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
         // P arrives in two halves (keys 0-63, then 64-127): the first half
         // of PV runs while the softmax finishes the second
         if (!wait_b(&bar_ph[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
-        if (!wait_b(&bar_vf[v % P2_NVS], (v / P2_NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
+        // both heads read the same V stage: head A's issue waited for it
+        if (x == 0 && !wait_b(&bar_vf[v % P2_NVS], (v / P2_NVS) & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA))
+          return false;
         tc_fence_after();
-        const uint32_t vaddr = sbase + GG::OFF_V + (v % P2_NVS) * GG::TB;
         const uint32_t pcol = tmem + (uint32_t)(x * 128);
         const uint32_t ocol = tmem + COL_O + (uint32_t)(x * D);
+        const uint32_t vlo = v0lo + (uint32_t)(v % P2_NVS) * (uint32_t)(GG::TB >> 4);
+        umma_ts_lh(ocol, pcol, vlo, vhi, GG::IDESC_PV, v > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), GG::IDESC_PV,
-                  (v > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 1; kk < 4; ++kk) umma_ts_lhc<1>(ocol, pcol + kk * 8, vlo + kk * 128, vhi, GG::IDESC_PV);
         if (!wait_b(&bar_pr[x], v & 1, &abort_flag, p.err, ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 4; kk < 8; ++kk)
-          umma_ts(ocol, pcol + kk * 8, desc_mn_sw128(vaddr + kk * 2048, HALF_BYTES), GG::IDESC_PV, 1u);
-        umma_commit(&bar_od[x]);
+        for (int kk = 4; kk < 8; ++kk) umma_ts_lhc<1>(ocol, pcol + kk * 8, vlo + kk * 128, vhi, GG::IDESC_PV);
+        if (v == n_all - 1) umma_commit(&bar_od[x]);  // the epilogue's wait: the last PV
         if (x == 1) umma_commit(&bar_ve[v % P2_NVS]);
         return true;
       };
@@ -1298,7 +1336,7 @@ bifocal_prefill2_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_con
       ++v;
     }
     // ---- epilogue: exactly one PV (the last) can be outstanding
-    if (ok && v > 0) ok = __all_sync(0xffffffffu, wait_b(&bar_od[hx], (v - 1) & 1, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
+    if (ok && v > 0) ok = __all_sync(0xffffffffu, wait_b(&bar_od[hx], 0, &abort_flag, p.err, ERR_TIMEOUT_SOFTMAX));
     if (ok) {
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
