@@ -194,6 +194,7 @@ BALANCE = [
     (tuple(range(300, 300 + 18 * 700, 700)), 16, 8, 128),      # 144 pairs: one unit per pair
     (tuple(range(50, 50 + 37 * 97, 97)), 16, 4, 128),          # 148 pairs: the (split, head, sequence) grid
     ((3000,) * 5 + (1,), 8, 1, 128),                           # one kv head: up to 148 units
+    (tuple(range(1, 1 + 70 * 37, 37)), 4, 2, 128),             # 70 sequences: the plan's chunks of 32
 ]
 
 
